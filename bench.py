@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Throughput of the fused ZeRO-DP shard step on B200.
+
+Default workload: GPT-2 1.5B-shaped parameters (48 layers, d = 1600, vocab
+50257: Psi = 1,557,611,200) at data-parallel degree Nd = 8, stage-2 layout
+(every simulated rank holds a full fp16 gradient), AdamW (wd 0.01), loss
+scale 65536, speculative mode.  One step = the whole hot path over all
+Nd owners: reduce-scatter sum of the 8 contributions, unscale, overflow check,
+Adam on the fp32 master/momentum/variance and the fp16 cast into the
+all-gathered parameter buffer.
+
+Prints one JSON line (rank 0).  ``value`` is owned parameters updated per
+second over all ranks with inputs resident in HBM; ``e2e`` repeats the
+measurement through the C-ABI call with the step's gradients copied from
+pinned host memory every step and the step result read back; ``roofline``
+reports the update kernel's algorithmic bytes per launch over its CUDA-event
+duration against the measured HBM copy bandwidth; ``cpu_baseline`` times the
+CPU oracle on a bounded sample on this host.
+
+Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): the path has
+no data exchange on one GPU, so N ranks run independent replicas (weak
+scaling); the only collectives are the timing barrier and the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused ZeRO shard-step params/s and achieved HBM GB/s (fraction of B200 peak)"
+UNIT = "params/s"
+FALLBACK_HBM_GBS = 6650.0  # used only if MEASURED_PEAKS.json is absent
+
+
+def _workloads():
+    from zero_dp_partitioned_shard_b200 import binding as B
+    from zero_dp_partitioned_shard_b200 import synth
+    return {
+        "gpt2-1.5b-stage2-nd8": dict(
+            desc="GPT-2 1.5B-shaped (48L d1600 vocab 50257, Psi=1,557,611,200), stage 2, Nd=8, "
+                 "AdamW wd 0.01, loss scale 65536, speculative mode",
+            sizes=synth.gpt2_xl_tensor_sizes, nd=8, stage=2, align=256, bucket=0, S=65536.0,
+            wd=0.01, clip=0.0, mode=B.ZERO_MODE_SPECULATIVE, layout=B.ZERO_GRADS_FULL,
+            owner_first=0, owner_count=None),
+        "24l-d2048-stage2-nd16-clip": dict(
+            desc="24-layer d2048 transformer (Psi=1,315,723,264), stage 2, Nd=16, 25M-element "
+                 "buckets, global-norm clip 1.0, loss scale 65536, stash mode",
+            sizes=synth.transformer_24l_d2048_tensor_sizes, nd=16, stage=2, align=256,
+            bucket=25_000_000, S=65536.0, wd=0.0, clip=1.0, mode=B.ZERO_MODE_STASH,
+            layout=B.ZERO_GRADS_FULL, owner_first=0, owner_count=None),
+        "7.5b-nd64-stage3-owner0": dict(
+            desc="stage-3 one-rank view of 7.5B params at Nd=64: owner 0's shard "
+                 "(L=117,187,584) with 64 fp16 contributions, speculative mode",
+            sizes=None, psi=7_500_000_000, nd=64, stage=3, align=256, bucket=0, S=1.0, wd=0.0,
+            clip=0.0, mode=B.ZERO_MODE_SPECULATIVE, layout=B.ZERO_GRADS_PER_OWNER,
+            owner_first=0, owner_count=1),
+    }
+
+
+def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
+    """(algorithmic, moved-by-mode) bytes per owned parameter of one step."""
+    alg = 2 * nd + 26  # Nd fp16 reads, master/m/v read+write (24), fp16 write (2)
+    moved = {0: alg, 1: 4 * nd + 26, 2: 2 * nd + 34}[mode]
+    return alg, moved
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+class Bench:
+    """Device buffers and the C-ABI arguments of one workload on one GPU."""
+
+    def __init__(self, wl: dict, psi_override: int | None, seed: int):
+        import torch
+        from zero_dp_partitioned_shard_b200 import binding as B
+        from zero_dp_partitioned_shard_b200 import synth
+        self.B, self.torch = B, torch
+        sizes = wl["sizes"]() if wl.get("sizes") else None
+        psi = psi_override or (sum(sizes) if sizes else wl["psi"])
+        if psi_override:
+            sizes = None
+        self.wl, self.psi, self.nd = wl, psi, wl["nd"]
+        self.plan = B.zero_plan(psi, self.nd, stage=wl["stage"], align_elems=wl["align"],
+                                bucket_elems=wl["bucket"], tensor_sizes=sizes)
+        info = B.zero_plan_query(self.plan)
+        L = self.L = info.shard_len
+        o0 = wl["owner_first"]
+        oc = self.nd if wl["owner_count"] is None else wl["owner_count"]
+        self.o0, self.oc = o0, oc
+        lo, hi = o0 * L, min((o0 + oc) * L, psi)
+        self.owned = hi - lo
+        n_state = oc * L
+        dev = torch.device("cuda")
+        spec = wl["mode"] == B.ZERO_MODE_SPECULATIVE
+        # gradient contributions
+        if wl["layout"] == B.ZERO_GRADS_FULL:
+            stride = info.psi_pad
+            self.grads = torch.empty(self.nd * stride, dtype=torch.float16, device=dev)
+            for r in range(self.nd):
+                row = self.grads[r * stride:(r + 1) * stride]
+                synth.fill_normal_(row[:psi], seed=seed * 1000 + r, std=1e-3, scale=wl["S"])
+                row[psi:].zero_()
+        else:
+            stride = L
+            self.grads = torch.empty(oc * self.nd * L, dtype=torch.float16, device=dev)
+            synth.fill_normal_(self.grads, seed=seed * 1000, std=1e-3, scale=wl["S"])
+        self.stride = stride
+        self.grad_bytes = self.grads.numel() * 2
+        f32 = lambda: torch.zeros(n_state, dtype=torch.float32, device=dev)
+        self.master = [synth.fill_normal_(f32(), seed=seed * 1000 + 999, std=0.02),
+                       f32() if spec else None]
+        self.exp_avg = [f32(), f32() if spec else None]
+        self.exp_avg_sq = [f32(), f32() if spec else None]
+        self.stash = f32() if wl["mode"] == B.ZERO_MODE_STASH else None
+        self.params = torch.zeros(psi, dtype=torch.float16, device=dev)
+        stream = torch.cuda.current_stream().cuda_stream
+        B.zero_cast_params(self.plan, self.master[0].data_ptr(), self.params.data_ptr(), o0, oc, stream)
+        self.opt_state = torch.zeros(B.OPT_STATE_BYTES, dtype=torch.uint8, device=dev)
+        self.result = torch.zeros(B.RESULT_BYTES, dtype=torch.uint8, device=dev)
+        B.zero_opt_state_init(self.opt_state.data_ptr(), stream)
+        self.hp = B.hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
+                            loss_scale=wl["S"], max_grad_norm=wl["clip"], mode=wl["mode"])
+        ptr = lambda t: t.data_ptr() if t is not None else 0
+        self.args = B.step_args(
+            grads=self.grads.data_ptr(), grad_rank_stride=stride, grad_layout=wl["layout"],
+            owner_first=o0, owner_count=oc, master=tuple(ptr(t) for t in self.master),
+            exp_avg=tuple(ptr(t) for t in self.exp_avg),
+            exp_avg_sq=tuple(ptr(t) for t in self.exp_avg_sq), params=self.params.data_ptr(),
+            grad_stash=ptr(self.stash), opt_state=self.opt_state.data_ptr(),
+            result=self.result.data_ptr())
+        ws_bytes = B.zero_workspace_bytes(self.plan, self.hp, self.args)
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        self.args.workspace = self.workspace.data_ptr()
+        self.args.workspace_bytes = ws_bytes
+        self.stream = stream
+        torch.cuda.synchronize()
+
+    def step(self, events=None):
+        if events is not None:
+            self.args.timing_events[0] = events[0].cuda_event
+            self.args.timing_events[1] = events[1].cuda_event
+        else:
+            self.args.timing_events[0] = None
+            self.args.timing_events[1] = None
+        self.B.zero_shard_step(self.plan, self.hp, self.args, self.stream)
+
+    def close(self):
+        self.B.zero_plan_destroy(self.plan)
+
+
+def _dist():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_baseline(wl: dict, budget_s: float, sample_psi: int, threads: int) -> dict:
+    """The CPU oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    from zero_dp_partitioned_shard_b200 import synth
+    nd = wl["nd"]
+    G = synth.grads_f16(nd, sample_psi, seed=5, std=1e-3, scale=wl["S"])
+    master = synth.normal_f32(sample_psi, seed=6, std=0.02)
+    m = np.zeros(sample_psi, np.float32)
+    v = np.zeros(sample_psi, np.float32)
+    P = np.zeros(sample_psi, np.uint16)
+    hp = oracle.HP(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
+                   loss_scale=wl["S"], max_grad_norm=wl["clip"])
+    opt = oracle.Opt()
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.step(G, master, m, v, P, hp, opt, threads=threads)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    alg, _ = bytes_per_param(nd, 0)
+    return {"value": sample_psi * steps / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{steps} oracle steps over {sample_psi:,} params x Nd={nd} "
+                      f"(same hyper-parameters), {el:.1f} s, OpenMP threads={threads}",
+            "gbs_alg": sample_psi * steps * alg / el / 1e9}
+
+
+def run_reference(args, wl_name: str, wl: dict):
+    """Reference arm: the CPU oracle timed on this host, on bounded samples."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from zero_dp_partitioned_shard_b200 import synth
+    threads = oracle.host_threads()
+    nd = wl["nd"]
+    sample = args.ref_sample
+    G = synth.grads_f16(nd, sample, seed=5, std=1e-3, scale=wl["S"])
+    master = synth.normal_f32(sample, seed=6, std=0.02)
+    m = np.zeros(sample, np.float32)
+    v = np.zeros(sample, np.float32)
+    P = np.zeros(sample, np.uint16)
+    hp = oracle.HP(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
+                   loss_scale=wl["S"], max_grad_norm=wl["clip"])
+    opt = oracle.Opt()
+    for _ in range(args.warmup):
+        oracle.step(G, master, m, v, P, hp, opt, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.step(G, master, m, v, P, hp, opt, threads=threads)
+    el = time.perf_counter() - t0
+    value = sample * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl_name, "description": wl["desc"], "psi": _psi_of(wl),
+                   "nd": nd, "sample_params_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} steps over {sample:,} params x Nd={nd}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _psi_of(wl):
+    return sum(wl["sizes"]()) if wl.get("sizes") else wl["psi"]
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gpt2-1.5b-stage2-nd8")
+    ap.add_argument("--psi", type=int, default=0, help="smaller Psi of the same workload (profiling)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 22)
+    ap.add_argument("--ref-sample", type=int, default=1 << 21)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wls = _workloads()
+    if args.workload not in wls:
+        ap.error(f"unknown workload {args.workload}; choose from {sorted(wls)}")
+    wl = wls[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, args.workload, wl)
+
+    import torch
+    from zero_dp_partitioned_shard_b200 import binding as B
+    world, rank, local = _dist()
+    bench = Bench(wl, args.psi or None, seed=1 + rank)
+    alg, moved = bytes_per_param(wl["nd"], wl["mode"])
+
+    # --- device-resident timing ---
+    for _ in range(args.warmup):
+        bench.step()
+    k_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+    for a, b in k_events:   # create the CUDA events before handing their handles over
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = B.zero_launch_count()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for k in range(args.steps):
+        bench.step(k_events[k])
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = B.zero_launch_count() - launches0
+    clk = clocks.stop()
+    _barrier(world)
+    ms = t_start.elapsed_time(t_end)
+    ms_max = _max_over_ranks(ms, world)
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in k_events)
+    k_ms_max = _max_over_ranks(k_ms, world)
+    value = world * bench.owned * args.steps / (ms_max / 1e3)
+    res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
+
+    # --- end to end through the C ABI, host buffers ---
+    e2e = None
+    if not args.no_e2e:
+        import psutil
+        need = bench.grad_bytes
+        if psutil.virtual_memory().available > 2.5 * need:
+            g_host = torch.empty(bench.grads.numel(), dtype=torch.float16, pin_memory=True)
+            g_host.copy_(bench.grads)
+            r_host = torch.empty(B.RESULT_BYTES, dtype=torch.uint8, pin_memory=True)
+            torch.cuda.synchronize()
+            for it in range(1 + args.e2e_steps):
+                if it == 1:
+                    _barrier(world)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                bench.grads.copy_(g_host, non_blocking=True)
+                bench.step()
+                r_host.copy_(bench.result, non_blocking=True)
+                torch.cuda.current_stream().synchronize()
+                B.step_result_from_bytes(r_host.numpy().tobytes())  # the caller reads the result
+            e1.record()
+            torch.cuda.synchronize()
+            e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
+            e2e = {"value": world * bench.owned * args.e2e_steps / (e_ms / 1e3), "unit": UNIT,
+                   "h2d_bytes_per_step": bench.grad_bytes, "d2h_bytes_per_step": B.RESULT_BYTES,
+                   "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps}
+            del g_host
+        else:
+            e2e = {"value": None, "unit": UNIT, "skipped": "host memory below 2.5x the gradient bytes"}
+
+    peak, peak_kind = measured_hbm_peak()
+    achieved = bench.owned * alg / (k_ms_max / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "description": wl["desc"], "psi": bench.psi,
+                   "nd": wl["nd"], "stage": wl["stage"], "owned_params_per_gpu": bench.owned,
+                   "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
+                   "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
+                   "step_gbs_alg": bench.owned * alg / (ms_max / args.steps / 1e3) / 1e9,
+                   "l2": "inputs larger than L2 (no flush): "
+                         f"{bench.owned * moved / 1e9:.1f} GB moved per step",
+                   "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "zs_update_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "kernel_ms": k_ms_max,
+                     "alg_bytes_per_launch": bench.owned * alg},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "last_step": {"overflow": res.overflow, "t": res.t},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.cpu_sample,
+                                            oracle.host_threads())
+    bench.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

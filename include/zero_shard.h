@@ -1,0 +1,304 @@
+/*
+ * zero_shard.h -- C ABI of libzero_shard.so, the B200 (sm_100a) ZeRO-DP
+ * partitioned mixed-precision Adam shard step.
+ *
+ * What ZeRO-DP does, and so what this library computes:
+ *   Each of Nd data-parallel processes owns one 1/Nd slice of the model state
+ *   (fp32 master copy, Adam momentum and variance; stage 2 also the gradient,
+ *   stage 3 also the fp16 parameters).  A reduce-scatter brings each owner the
+ *   summed gradient of its slice, the owner updates only its slice, and an
+ *   all-gather rebuilds the full fp16 parameters.
+ *   Sources: anthology-of-the-sota note 103 on ZeRO (dmarx.github.io),
+ *   sections "Method" and "Concepts"; "ZeRO memory optimization: training
+ *   large models" (trishampatil.com), sections "ZeRO-1", "ZeRO-2", "ZeRO-3"
+ *   and "Forward/Backward Under ZeRO-3"; "ZeRO: partitioning training state
+ *   across GPUs" (upskillscore.com), section "How it works".
+ *
+ * On one GPU the Nd ranks are simulated: their fp16 gradient contributions
+ * sit side by side in device memory and one fused kernel per call sums them
+ * (the reduce-scatter), unscales by the loss scale, checks for inf/NaN,
+ * optionally clips by the global L2 norm, applies Adam/AdamW to the owned
+ * fp32 state and writes the fp16 cast straight into the full parameter
+ * buffer at the owner's offset (the all-gather layout).
+ *
+ * Arithmetic (the pages give no update equations; textbook readings):
+ *   s_i  = c_0,i + c_1,i + ... + c_{Nd-1},i      fp32, left to right by rank
+ *   g_i  = s_i * (fp32)(1/S)      [(fp32)(1/(S*Nd)) when averaging]
+ *   skip the whole step if any g_i (i < Psi, pads excluded) is not finite
+ *   norm = sqrt(sum_i (double)g_i^2); c = max/norm if norm > max else 1
+ *   g^_i = g_i * c
+ *   m = b1*m + (1-b1)*g^;  v = b2*v + (1-b2)*(g^*g^)
+ *   p = (p - (lr*wd)*p) - lr*((m/bc1)/(sqrt(v/bc2) + eps))
+ *   bc_k = (fp32)(1 - b_k^t), b_k^t kept as fp64 running products
+ *   P_i = fp16 round-to-nearest-even of p
+ * (Kingma & Ba 2015, Alg. 1; decoupled decay per Loshchilov & Hutter 2019.)
+ * Every fp32 operation above is one IEEE-rounded operation (no fused
+ * multiply-add), so results are deterministic and independent of the launch
+ * geometry; only the norm's fp64 summation order depends on it.
+ *
+ * Conventions for every call:
+ *   - Pointers documented "device" are CUDA device addresses on the device
+ *     current when the call is made; "host" pointers are ordinary memory.
+ *   - fp16 data is IEEE binary16 passed as void* / uint16_t bit patterns.
+ *   - The caller allocates and owns every device buffer (parameters, state,
+ *     gradients, workspace).  The library allocates only the host-side plan
+ *     object, never device memory, and never synchronises a stream.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All device work of a call is enqueued on it, in order.
+ *   - Arguments are validated before anything is launched; a failed check
+ *     returns a non-zero status and enqueues nothing.  zero_last_error()
+ *     then describes the failure (per calling thread).
+ *   - A gradient overflow is NOT an error: the call returns ZERO_OK and the
+ *     device-side result records overflow = 1.
+ */
+#ifndef ZERO_SHARD_H
+#define ZERO_SHARD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZERO_SHARD_ABI_VERSION 1
+
+/* Every entry point is exported with default visibility; the library hides
+ * everything else. */
+#if defined(__GNUC__)
+#define ZERO_API __attribute__((visibility("default")))
+#else
+#define ZERO_API
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+typedef int32_t zero_status;
+#define ZERO_OK 0
+#define ZERO_ERR_INVALID_ARG 1 /* null / out-of-range argument, bad combination */
+#define ZERO_ERR_ALIGNMENT 2   /* a pointer is not aligned to its element size  */
+#define ZERO_ERR_CUDA 3        /* a CUDA runtime call or launch failed          */
+#define ZERO_ERR_WORKSPACE 4   /* workspace missing or smaller than required    */
+#define ZERO_ERR_TIMEOUT 5     /* reserved: no kernel of this library waits     */
+#define ZERO_ERR_UNSUPPORTED 6 /* combination not available (e.g. clip + speculative) */
+
+/* ---- enumerations --------------------------------------------------------- */
+/* Skip-correct execution modes of zero_shard_step (overflow must be known
+ * before any state changes):
+ *   SPECULATIVE: one fused pass reads the live state slot and writes the other
+ *     (ping-pong master/m/v); the slot index flips only if no overflow was
+ *     seen, and on overflow the fp16 parameters are re-cast from the live
+ *     master.  Minimal traffic (2*Nd + 26 bytes per owned parameter), +12
+ *     bytes of memory per parameter.  No clipping.
+ *   TWO_PASS: a statistics pass (overflow flag, norm) re-reads the gradients
+ *     before the in-place update.  4*Nd + 26 bytes per parameter, no extra
+ *     memory.
+ *   STASH: the statistics pass also writes the reduced fp32 gradient to a
+ *     caller buffer and the in-place update reads it back.  2*Nd + 34 bytes
+ *     per parameter, +4 bytes of memory per parameter. */
+#define ZERO_MODE_SPECULATIVE 0
+#define ZERO_MODE_TWO_PASS 1
+#define ZERO_MODE_STASH 2
+
+/* Layout of the gradient contributions:
+ *   FULL (stages 1 and 2: every rank holds a full-size gradient): rank r's
+ *     contribution to flat parameter j is grads[r * grad_rank_stride + j],
+ *     grad_rank_stride >= psi.
+ *   PER_OWNER (stage 3: contributions arrive already partitioned): rank r's
+ *     contribution to element i of owner (owner_first + k) is
+ *     grads[(k * nd + r) * grad_rank_stride + i], grad_rank_stride >= L
+ *     (0 means L). */
+#define ZERO_GRADS_FULL 0
+#define ZERO_GRADS_PER_OWNER 1
+
+/* ---- plan ------------------------------------------------------------------ */
+/* Partition of Psi parameters over Nd owners ("ZeRO memory optimization",
+ * trishampatil.com, sections "ZeRO-1/2/3"; upskillscore.com guide, "How it
+ * works").  Every owner gets a slice of the same padded length
+ * L = ceil(Psi / (Nd * A)) * A elements, so shard starts are A-aligned and
+ * only the last non-empty shard is short of real elements; pads are never
+ * read as data and never written to the parameters.  Buckets are the fixed
+ * B-element ranges [k*B, min((k+1)*B, Psi)) of the flat buffer in which the
+ * reduce-scatter is issued (the constant-size fused buffers of ZeRO-R,
+ * anthology-of-the-sota note 103, "Method"). */
+typedef struct zero_plan_desc {
+    int64_t psi;                 /* parameters, >= 1 */
+    int64_t align_elems;         /* A >= 1 (256 is the usual choice) */
+    int64_t bucket_elems;        /* B >= 0; 0 = one bucket holding everything */
+    const int64_t* tensor_sizes; /* host, optional: tensors laid back to back; must sum to psi */
+    int32_t nd;                  /* data-parallel degree, >= 1 */
+    int32_t stage;               /* 0 (plain DP, accounting only), 1, 2 or 3 */
+    int32_t n_tensors;           /* entries in tensor_sizes (0 if NULL) */
+    int32_t reserved;            /* must be 0 */
+} zero_plan_desc;
+
+typedef struct zero_plan_s zero_plan_t; /* opaque, host only */
+
+typedef struct zero_plan_info {
+    int64_t psi, psi_pad, shard_len, align_elems, bucket_elems, n_buckets, n_segments;
+    int32_t nd, stage;
+} zero_plan_info;
+
+/* One piece of a tensor held by one owner (a tensor can straddle owners). */
+typedef struct zero_segment {
+    int64_t tensor, owner, offset_in_tensor, length, offset_in_shard;
+} zero_segment;
+
+/* Builds the plan (host only, no device touched).  *out must later be
+ * released with zero_plan_destroy.  Errors: INVALID_ARG for psi < 1, nd < 1,
+ * A < 1, B < 0, stage outside 0..3, or tensor sizes that do not sum to psi. */
+ZERO_API zero_status zero_plan(const zero_plan_desc* desc, zero_plan_t** out);
+ZERO_API zero_status zero_plan_query(const zero_plan_t* plan, zero_plan_info* out);
+/* Owner's flat range [start, start + real_len), 0 <= real_len <= L. */
+ZERO_API zero_status zero_plan_shard(const zero_plan_t* plan, int32_t owner, int64_t* start, int64_t* real_len);
+/* Bucket k's flat range, 0 <= k < n_buckets. */
+ZERO_API zero_status zero_plan_bucket(const zero_plan_t* plan, int64_t k, int64_t* start, int64_t* len);
+/* Copies up to cap tensor pieces (tensor order, then owner order) into out
+ * (host); *n_out receives the total number.  out may be NULL when cap == 0. */
+ZERO_API zero_status zero_plan_segments(const zero_plan_t* plan, zero_segment* out, int64_t cap, int64_t* n_out);
+ZERO_API void zero_plan_destroy(zero_plan_t* plan);
+
+/* ---- accounting --------------------------------------------------------------- */
+/* Model-state bytes per device and communication volume per step.
+ * "ZeRO memory optimization" (trishampatil.com): "The Real Problem" (2 Psi
+ * fp16 params + 2 Psi fp16 grads + 12 Psi fp32 Adam state = 16 Psi) and the
+ * table under "The Full Progression, in One View": stage 0 (plain DP) 16 Psi,
+ * stage 1 4 Psi + 12 Psi/Nd, stage 2 2 Psi + 14 Psi/Nd, stage 3 16 Psi/Nd;
+ * communication 2 Psi, 2 Psi, 2 Psi, 3 Psi elements per process per step
+ * (stage 3 adds a second parameter all-gather, upskillscore.com guide, "How
+ * it works").  The *_padded fields replace Psi/Nd by the padded shard length
+ * L of alignment A; comm_bytes counts 2 bytes per fp16 element;
+ * comm_elems_ring ((Nd-1)/Nd of each collective) is a derived extra. */
+typedef struct zero_state_report {
+    double params_bytes, grads_bytes, optim_bytes, total_bytes;
+    int64_t params_bytes_padded, grads_bytes_padded, optim_bytes_padded, total_bytes_padded;
+    double reduction;       /* 16 Psi / total_bytes */
+    double comm_elems;      /* per process per step */
+    double comm_bytes;
+    double comm_elems_ring;
+} zero_state_report;
+
+ZERO_API zero_status zero_state_bytes(int64_t psi, int32_t nd, int32_t stage, int64_t align_elems,
+                             zero_state_report* out);
+
+/* ---- device-side state -------------------------------------------------------- */
+/* Optimizer bookkeeping, resident in device memory (caller allocates >= 64
+ * bytes, 8-byte aligned; zero_opt_state_init fills it).  Only the library's
+ * kernels update it, so a step never needs a host synchronisation. */
+typedef struct zero_opt_state {
+    int64_t t;        /* steps applied (skipped steps do not count) */
+    double beta1_pow; /* beta1^t, fp64 running product */
+    double beta2_pow; /* beta2^t */
+    int64_t skipped;  /* steps skipped on overflow */
+    int32_t cur;      /* SPECULATIVE: ping-pong slot (0/1) holding the live state */
+    int32_t reserved;
+} zero_opt_state;
+
+/* Per-call outcome, written to device memory when args->result != NULL. */
+typedef struct zero_step_result {
+    double grad_norm;  /* global L2 norm of the unscaled reduced gradient;
+                          NaN in SPECULATIVE mode and on overflow */
+    int64_t t;         /* zero_opt_state.t after the call */
+    int64_t skipped;   /* zero_opt_state.skipped after the call */
+    float clip_coef;   /* coefficient applied (1 when not clipping) */
+    int32_t overflow;  /* 1: a non-finite gradient was seen, nothing was updated */
+} zero_step_result;
+
+/* ---- the step ---------------------------------------------------------------------- */
+typedef struct zero_hparams {
+    float lr, beta1, beta2, eps, weight_decay;
+    float loss_scale;      /* S > 0; contributions carry the loss scaled by S */
+    float max_grad_norm;   /* > 0: clip to this global norm; <= 0: no clipping */
+    int32_t average_over_nd; /* 1: divide the sum by Nd as well */
+    int32_t mode;          /* ZERO_MODE_* */
+    int32_t reserved;      /* must be 0 */
+} zero_hparams;
+
+/* Buffers of one call.  The call updates owners owner_first ..
+ * owner_first + owner_count - 1 (all Nd owners of a plan: the whole simulated
+ * data-parallel group; one owner: a single rank's view).
+ *   master/exp_avg/exp_avg_sq[k]: device fp32.  Element i of owner
+ *     (owner_first + j) lives at [j * L + i]; only i < real_len is touched.
+ *     Slot [1] is required by SPECULATIVE only (and ignored otherwise).
+ *     16-byte aligned pointers take the vectorised path.
+ *   params: device fp16, the full assembled buffer of psi elements: owner o
+ *     writes params[o * L + i].  Positions of other owners are untouched.
+ *   grads: device fp16 contributions in grad_layout (ZERO_GRADS_*).
+ *   grad_stash: STASH mode only: device fp32 laid out like master.
+ *   opt_state: device zero_opt_state; result: device zero_step_result or NULL.
+ *   workspace: device scratch of at least zero_workspace_bytes() bytes,
+ *     256-byte aligned; contents need no initialisation and are clobbered.
+ *   timing_events: optional pair of cudaEvent_t (as void*) recorded on the
+ *     stream immediately before and after the parameter-update kernel(s), so
+ *     a caller can time the dominant kernel alone; NULL entries = none. */
+typedef struct zero_step_args {
+    const void* grads;
+    int64_t grad_rank_stride;
+    int32_t grad_layout;
+    int32_t owner_first;
+    int32_t owner_count;
+    int32_t reserved;
+    float* master[2];
+    float* exp_avg[2];
+    float* exp_avg_sq[2];
+    void* params;
+    float* grad_stash;
+    void* opt_state;
+    void* result;
+    void* workspace;
+    size_t workspace_bytes;
+    void* timing_events[2];
+} zero_step_args;
+
+/* Writes {t = 0, beta1_pow = beta2_pow = 1, skipped = 0, cur = 0} into the
+ * device zero_opt_state at opt_state, on stream. */
+ZERO_API zero_status zero_opt_state_init(void* opt_state, void* stream);
+
+/* Bytes of scratch a zero_shard_step call with these arguments needs (the
+ * workspace fields of args are ignored).  A few hundred bytes in SPECULATIVE
+ * mode; in TWO_PASS / STASH also 16 KiB of fp64 norm partials per bucket. */
+ZERO_API zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hparams* hp,
+                                 const zero_step_args* args, size_t* bytes);
+
+/* One ZeRO-DP step for the owners in args (reduce-scatter sum + unscale +
+ * overflow check + optional clip + Adam + fp16 cast into the all-gather
+ * layout), enqueued on stream without host synchronisation.  On overflow
+ * nothing changes: master/m/v, params (see SPECULATIVE note below) and
+ * opt_state.t keep their values and opt_state.skipped grows by one.
+ * SPECULATIVE note: on a skipped step params is rewritten as the fp16 cast of
+ * the unchanged live master, which equals its previous contents whenever
+ * params holds that cast (true after any step of this library, and after
+ * zero_cast_params).
+ * The overflow flag and the norm are global over every owner of the call.
+ * Errors: INVALID_ARG (null pointers, owner range outside the plan, bad
+ * hyper-parameters or layout), ALIGNMENT (pointer not aligned to its element
+ * size), UNSUPPORTED (clipping in SPECULATIVE mode), WORKSPACE, CUDA. */
+ZERO_API zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
+                            const zero_step_args* args, void* stream);
+
+/* Gather-assembly (the stage-3 all-gather seen by one rank): for every owner
+ * r whose shard_ptrs[r] (host array of nd device pointers) is not NULL,
+ * copies its fp16 shard [0, real_len_r) into params_full[r * L ...].
+ * "ZeRO memory optimization" (trishampatil.com), "Forward/Backward Under
+ * ZeRO-3": a process gathers the parameter shards it does not own. */
+ZERO_API zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard_ptrs,
+                               void* params_full, void* stream);
+
+/* params[(owner_first + j) * L + i] = fp16(master[j * L + i]) for the owners
+ * owner_first .. owner_first + owner_count - 1: establishes the fp16 copy
+ * of a freshly initialised fp32 master (device pointers). */
+ZERO_API zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,
+                             int32_t owner_first, int32_t owner_count, void* stream);
+
+/* ---- diagnostics ---------------------------------------------------------------- */
+ZERO_API int32_t zero_abi_version(void);
+ZERO_API const char* zero_strerror(zero_status status);
+/* Message of the last failed call on this thread ("" if none). */
+ZERO_API const char* zero_last_error(void);
+/* Number of kernels this library has launched in this process. */
+ZERO_API uint64_t zero_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_SHARD_H */

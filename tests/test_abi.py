@@ -1,0 +1,244 @@
+"""C-ABI checks that need no GPU: the library loads and exports every
+function include/*.h declares, the ctypes structs match the C layout, the
+host planner and accounting agree bit for bit with the oracle, and invalid
+arguments are rejected before anything is launched."""
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from zero_dp_partitioned_shard_b200 import binding as B
+from zero_dp_partitioned_shard_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(zero_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert {"zero_plan", "zero_shard_step", "zero_gather_params", "zero_state_bytes"} <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = declared - exported
+    assert not missing, f"declared but not exported: {sorted(missing)}"
+    # the binding covers exactly the declared surface
+    assert set(B.SIGNATURES) == declared
+    lib = B.lib()
+    for name in declared:
+        assert getattr(lib, name) is not None
+    assert B.zero_abi_version() == 1
+    # nothing else leaks out of the library (hidden visibility)
+    assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
+
+
+_LAYOUT_PROBE = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "zero_shard.h"
+#define S(T) printf(#T " %zu\n", sizeof(T));
+#define O(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+  S(zero_plan_desc) S(zero_plan_info) S(zero_segment) S(zero_state_report)
+  S(zero_opt_state) S(zero_step_result) S(zero_hparams) S(zero_step_args)
+  O(zero_step_args, master) O(zero_step_args, params) O(zero_step_args, workspace_bytes)
+  O(zero_step_args, timing_events) O(zero_hparams, mode) O(zero_opt_state, cur)
+  O(zero_step_result, overflow) O(zero_plan_desc, nd) O(zero_plan_info, nd)
+  return 0;
+}
+"""
+
+
+def test_ctypes_structs_match_the_c_header(tmp_path):
+    src = tmp_path / "probe.c"
+    src.write_text(_LAYOUT_PROBE)
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = dict(line.rsplit(" ", 1) for line in subprocess.run([str(exe)], capture_output=True,
+                                                             text=True, check=True).stdout.split("\n") if line)
+    got = {k: int(v) for k, v in got.items()}
+    py = {"zero_plan_desc": B.PlanDesc, "zero_plan_info": B.PlanInfo, "zero_segment": B.Segment,
+          "zero_state_report": B.StateReport, "zero_opt_state": B.OptState,
+          "zero_step_result": B.StepResult, "zero_hparams": B.HParams, "zero_step_args": B.StepArgs}
+    for cname, ctype in py.items():
+        assert got[cname] == C.sizeof(ctype), cname
+    for key, val in got.items():
+        if "." in key:
+            cname, field = key.split(".")
+            assert getattr(py[cname], field).offset == val, key
+    assert got["zero_opt_state"] <= B.OPT_STATE_BYTES and got["zero_step_result"] <= B.RESULT_BYTES
+
+
+def _plan_cases():
+    rs = np.random.default_rng(5)
+    cases = [(1, 1, 1, 0), (7, 3, 1, 0), (1_000_003, 4, 256, 0), (1_000_003, 4, 256, 25_000),
+             (1_557_611_200, 8, 256, 0), (7_500_000_000, 64, 256, 0), (7_500_000_000, 64, 1, 0),
+             (1_315_723_264, 16, 256, 25_000_000), (5, 64, 8, 3)]
+    for _ in range(200):
+        cases.append((int(rs.integers(1, 100_000)), int(rs.integers(1, 70)),
+                      int(rs.choice([1, 2, 8, 16, 256])), int(rs.choice([0, 1, 7, 1000, 4096]))))
+    return cases
+
+
+def test_planner_matches_oracle_bit_exact():
+    for psi, nd, a, b in _plan_cases():
+        ref = oracle.plan(psi, nd, a, b)
+        h = B.zero_plan(psi, nd, stage=2, align_elems=a, bucket_elems=b)
+        try:
+            info = B.zero_plan_query(h)
+            assert (info.psi, info.psi_pad, info.shard_len, info.n_buckets) == \
+                   (ref.psi, ref.psi_pad, ref.shard_len, ref.n_buckets)
+            for r in sorted({0, nd - 1, nd // 2}):
+                assert B.zero_plan_shard(h, r) == ref.shard(r)
+            for k in sorted({0, ref.n_buckets - 1}):
+                assert B.zero_plan_bucket(h, k) == ref.bucket_range(k)
+        finally:
+            B.zero_plan_destroy(h)
+
+
+def test_segments_match_oracle():
+    rs = np.random.default_rng(8)
+    lists = [synth.transformer_24l_d2048_tensor_sizes(), synth.gpt2_xl_tensor_sizes()]
+    for _ in range(30):
+        lists.append([int(x) for x in rs.integers(0, 500, size=int(rs.integers(1, 20)))])
+    for sizes in lists:
+        psi = sum(sizes)
+        if psi == 0:
+            continue
+        for nd, a in ((16, 256), (8, 256), (3, 1), (7, 16)):
+            ref = oracle.plan(psi, nd, a).tensor_segments(sizes)
+            h = B.zero_plan(psi, nd, align_elems=a, tensor_sizes=sizes)
+            try:
+                got = np.array(B.zero_plan_segments(h), dtype=np.int64).reshape(-1, 5)
+                assert np.array_equal(got, ref)
+                assert B.zero_plan_query(h).n_segments == len(ref)
+            finally:
+                B.zero_plan_destroy(h)
+
+
+def test_state_bytes_matches_oracle_bit_exact():
+    for psi, nd, a, _ in _plan_cases()[:60]:
+        for stage in range(4):
+            got = B.zero_state_bytes(psi, nd, stage, a)
+            ref = oracle.state_bytes(psi, nd, stage, a)
+            for k, v in ref.items():
+                assert got[k] == v, (psi, nd, stage, a, k)
+
+
+@pytest.mark.parametrize("bad", [dict(psi=0, nd=1), dict(psi=10, nd=0), dict(psi=10, nd=2, stage=4),
+                                 dict(psi=10, nd=2, align_elems=0), dict(psi=10, nd=2, bucket_elems=-1),
+                                 dict(psi=10, nd=2, tensor_sizes=[3, 3])])
+def test_plan_rejects_bad_descriptions(bad):
+    with pytest.raises(B.ZeroError) as e:
+        B.zero_plan(**bad)
+    assert e.value.status == B.ZERO_ERR_INVALID_ARG
+
+
+# --- validation of zero_shard_step: every case below is rejected by host-side
+# checks before anything is launched (addresses are never dereferenced) ---
+
+FAKE = 1 << 40  # 256-byte aligned fake device address
+
+
+def _args(**kw):
+    base = dict(grads=FAKE, grad_rank_stride=1024, master=(FAKE, FAKE), exp_avg=(FAKE, FAKE),
+                exp_avg_sq=(FAKE, FAKE), params=FAKE, opt_state=FAKE, workspace=FAKE,
+                workspace_bytes=1 << 20, owner_first=0, owner_count=4)
+    base.update(kw)
+    return B.step_args(**base)
+
+
+@pytest.mark.parametrize("case,status", [
+    ("owner_range", B.ZERO_ERR_INVALID_ARG), ("owner_count0", B.ZERO_ERR_INVALID_ARG),
+    ("null_grads", B.ZERO_ERR_INVALID_ARG), ("null_slot1", B.ZERO_ERR_INVALID_ARG),
+    ("stride_small", B.ZERO_ERR_INVALID_ARG), ("bad_layout", B.ZERO_ERR_INVALID_ARG),
+    ("bad_mode", B.ZERO_ERR_INVALID_ARG), ("bad_scale", B.ZERO_ERR_INVALID_ARG),
+    ("bad_beta", B.ZERO_ERR_INVALID_ARG), ("clip_spec", B.ZERO_ERR_UNSUPPORTED),
+    ("stash_missing", B.ZERO_ERR_INVALID_ARG), ("misaligned_master", B.ZERO_ERR_ALIGNMENT),
+    ("misaligned_params", B.ZERO_ERR_ALIGNMENT), ("small_ws", B.ZERO_ERR_WORKSPACE),
+    ("null_ws", B.ZERO_ERR_WORKSPACE), ("misaligned_ws", B.ZERO_ERR_ALIGNMENT),
+    ("reserved", B.ZERO_ERR_INVALID_ARG),
+])
+def test_step_validation_rejects_before_launch(case, status):
+    plan = B.zero_plan(1000, 4, stage=1, align_elems=8)
+    hp = B.hparams(loss_scale=1024.0)
+    args = _args()
+    if case == "owner_range":
+        args = _args(owner_first=2, owner_count=3)
+    elif case == "owner_count0":
+        args = _args(owner_count=0)
+    elif case == "null_grads":
+        args = _args(grads=0)
+    elif case == "null_slot1":
+        args = _args(master=(FAKE, 0))
+    elif case == "stride_small":
+        args = _args(grad_rank_stride=999)
+    elif case == "bad_layout":
+        args = _args(grad_layout=7)
+    elif case == "bad_mode":
+        hp = B.hparams(loss_scale=1024.0, mode=9)
+    elif case == "bad_scale":
+        hp = B.hparams(loss_scale=0.0)
+    elif case == "bad_beta":
+        hp = B.hparams(loss_scale=1.0, beta2=1.0)
+    elif case == "clip_spec":
+        hp = B.hparams(loss_scale=1.0, max_grad_norm=1.0)
+    elif case == "stash_missing":
+        hp = B.hparams(loss_scale=1.0, mode=B.ZERO_MODE_STASH)
+    elif case == "misaligned_master":
+        args = _args(master=(FAKE + 2, FAKE))
+    elif case == "misaligned_params":
+        args = _args(params=FAKE + 1)
+    elif case == "small_ws":
+        args = _args(workspace_bytes=16)
+    elif case == "null_ws":
+        args = _args(workspace=0)
+    elif case == "misaligned_ws":
+        args = _args(workspace=FAKE + 16)
+    elif case == "reserved":
+        args = _args()
+        args.reserved = 1
+    before = B.zero_launch_count()
+    try:
+        with pytest.raises(B.ZeroError) as e:
+            B.zero_shard_step(plan, hp, args)
+        assert e.value.status == status, B.zero_last_error()
+        assert B.zero_last_error()
+    finally:
+        B.zero_plan_destroy(plan)
+    assert B.zero_launch_count() == before
+
+
+def test_workspace_bytes_per_mode():
+    plan = B.zero_plan(1_315_723_264, 16, stage=2, align_elems=256, bucket_elems=25_000_000)
+    try:
+        args = _args(grad_rank_stride=1_315_723_264, owner_count=16, grad_stash=FAKE)
+        spec = B.zero_workspace_bytes(plan, B.hparams(loss_scale=1.0), args)
+        two = B.zero_workspace_bytes(plan, B.hparams(loss_scale=1.0, mode=B.ZERO_MODE_TWO_PASS,
+                                                      max_grad_norm=1.0), args)
+        assert spec == 256
+        assert two == 256 + 53 * 2048 * 8
+    finally:
+        B.zero_plan_destroy(plan)
+
+
+def test_strerror_names_every_status():
+    for s in range(7):
+        assert B.zero_strerror(s) and "unknown" not in B.zero_strerror(s)
+    assert "unknown" in B.zero_strerror(99)

@@ -1,0 +1,290 @@
+"""ctypes binding of ``libzero_shard.so`` (declared in ``include/zero_shard.h``).
+
+Argument marshalling only: every function below has the name of the C entry
+point it calls, converts Python values / integer device addresses into the C
+structs, and raises :class:`ZeroError` (carrying the status code and the
+library's message) when the call returns a non-zero status.  All device work
+runs in the library's CUDA kernels; there is no Python or CPU fallback, and a
+missing library raises at first use.
+
+Device buffers are passed as integer addresses (``tensor.data_ptr()``) and
+streams / events as their raw handles (``torch.cuda.Stream.cuda_stream``,
+``torch.cuda.Event.cuda_event``), so this module does not depend on torch.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzero_shard.so")
+
+ZERO_OK = 0
+ZERO_ERR_INVALID_ARG = 1
+ZERO_ERR_ALIGNMENT = 2
+ZERO_ERR_CUDA = 3
+ZERO_ERR_WORKSPACE = 4
+ZERO_ERR_TIMEOUT = 5
+ZERO_ERR_UNSUPPORTED = 6
+
+ZERO_MODE_SPECULATIVE = 0
+ZERO_MODE_TWO_PASS = 1
+ZERO_MODE_STASH = 2
+
+ZERO_GRADS_FULL = 0
+ZERO_GRADS_PER_OWNER = 1
+
+OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (40 bytes used)
+RESULT_BYTES = 64      # device allocation for zero_step_result (32 bytes used)
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status: int, func: str, message: str):
+        super().__init__(f"{func}: status {status} ({message})")
+        self.status = status
+
+
+class PlanDesc(C.Structure):
+    _fields_ = [("psi", C.c_int64), ("align_elems", C.c_int64), ("bucket_elems", C.c_int64),
+                ("tensor_sizes", C.c_void_p), ("nd", C.c_int32), ("stage", C.c_int32),
+                ("n_tensors", C.c_int32), ("reserved", C.c_int32)]
+
+
+class PlanInfo(C.Structure):
+    _fields_ = [("psi", C.c_int64), ("psi_pad", C.c_int64), ("shard_len", C.c_int64),
+                ("align_elems", C.c_int64), ("bucket_elems", C.c_int64),
+                ("n_buckets", C.c_int64), ("n_segments", C.c_int64),
+                ("nd", C.c_int32), ("stage", C.c_int32)]
+
+
+class Segment(C.Structure):
+    _fields_ = [("tensor", C.c_int64), ("owner", C.c_int64), ("offset_in_tensor", C.c_int64),
+                ("length", C.c_int64), ("offset_in_shard", C.c_int64)]
+
+
+class StateReport(C.Structure):
+    _fields_ = [("params_bytes", C.c_double), ("grads_bytes", C.c_double),
+                ("optim_bytes", C.c_double), ("total_bytes", C.c_double),
+                ("params_bytes_padded", C.c_int64), ("grads_bytes_padded", C.c_int64),
+                ("optim_bytes_padded", C.c_int64), ("total_bytes_padded", C.c_int64),
+                ("reduction", C.c_double), ("comm_elems", C.c_double),
+                ("comm_bytes", C.c_double), ("comm_elems_ring", C.c_double)]
+
+
+class OptState(C.Structure):
+    _fields_ = [("t", C.c_int64), ("beta1_pow", C.c_double), ("beta2_pow", C.c_double),
+                ("skipped", C.c_int64), ("cur", C.c_int32), ("reserved", C.c_int32)]
+
+
+class StepResult(C.Structure):
+    _fields_ = [("grad_norm", C.c_double), ("t", C.c_int64), ("skipped", C.c_int64),
+                ("clip_coef", C.c_float), ("overflow", C.c_int32)]
+
+
+class HParams(C.Structure):
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
+                ("eps", C.c_float), ("weight_decay", C.c_float), ("loss_scale", C.c_float),
+                ("max_grad_norm", C.c_float), ("average_over_nd", C.c_int32),
+                ("mode", C.c_int32), ("reserved", C.c_int32)]
+
+
+class StepArgs(C.Structure):
+    _fields_ = [("grads", C.c_void_p), ("grad_rank_stride", C.c_int64),
+                ("grad_layout", C.c_int32), ("owner_first", C.c_int32),
+                ("owner_count", C.c_int32), ("reserved", C.c_int32),
+                ("master", C.c_void_p * 2), ("exp_avg", C.c_void_p * 2),
+                ("exp_avg_sq", C.c_void_p * 2), ("params", C.c_void_p),
+                ("grad_stash", C.c_void_p), ("opt_state", C.c_void_p), ("result", C.c_void_p),
+                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
+                ("timing_events", C.c_void_p * 2)]
+
+
+_lib = None
+_P = C.c_void_p
+_S = C.c_int32
+
+# name -> (restype, argtypes) of every exported symbol of include/zero_shard.h
+SIGNATURES = {
+    "zero_plan": (_S, [C.POINTER(PlanDesc), C.POINTER(_P)]),
+    "zero_plan_query": (_S, [_P, C.POINTER(PlanInfo)]),
+    "zero_plan_shard": (_S, [_P, C.c_int32, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
+    "zero_plan_bucket": (_S, [_P, C.c_int64, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]),
+    "zero_plan_segments": (_S, [_P, _P, C.c_int64, C.POINTER(C.c_int64)]),
+    "zero_plan_destroy": (None, [_P]),
+    "zero_state_bytes": (_S, [C.c_int64, C.c_int32, C.c_int32, C.c_int64, C.POINTER(StateReport)]),
+    "zero_opt_state_init": (_S, [_P, _P]),
+    "zero_workspace_bytes": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), C.POINTER(C.c_size_t)]),
+    "zero_shard_step": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
+    "zero_gather_params": (_S, [_P, _P, _P, _P]),
+    "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, _P]),
+    "zero_abi_version": (C.c_int32, []),
+    "zero_strerror": (C.c_char_p, [_S]),
+    "zero_last_error": (C.c_char_p, []),
+    "zero_launch_count": (C.c_uint64, []),
+}
+
+
+def lib() -> C.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python zero_dp_partitioned_shard_b200/build.py` "
+                "(there is no CPU fallback)")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        if L.zero_abi_version() != 1:
+            raise ImportError("libzero_shard.so ABI version mismatch")
+        _lib = L
+    return _lib
+
+
+def _check(status: int, func: str) -> None:
+    if status != ZERO_OK:
+        raise ZeroError(status, func, lib().zero_last_error().decode())
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def zero_plan(psi: int, nd: int, stage: int = 1, align_elems: int = 256, bucket_elems: int = 0,
+              tensor_sizes=None) -> int:
+    """Returns an opaque plan handle; release it with zero_plan_destroy."""
+    sizes = None
+    if tensor_sizes is not None:
+        sizes = (C.c_int64 * len(tensor_sizes))(*[int(x) for x in tensor_sizes])
+    d = PlanDesc(psi, align_elems, bucket_elems, C.cast(sizes, C.c_void_p) if sizes else None,
+                 nd, stage, len(tensor_sizes) if tensor_sizes is not None else 0, 0)
+    h = C.c_void_p()
+    _check(lib().zero_plan(C.byref(d), C.byref(h)), "zero_plan")
+    return h.value
+
+
+def zero_plan_query(plan: int) -> PlanInfo:
+    info = PlanInfo()
+    _check(lib().zero_plan_query(plan, C.byref(info)), "zero_plan_query")
+    return info
+
+
+def zero_plan_shard(plan: int, owner: int) -> tuple[int, int]:
+    s, n = C.c_int64(), C.c_int64()
+    _check(lib().zero_plan_shard(plan, owner, C.byref(s), C.byref(n)), "zero_plan_shard")
+    return s.value, n.value
+
+
+def zero_plan_bucket(plan: int, k: int) -> tuple[int, int]:
+    s, n = C.c_int64(), C.c_int64()
+    _check(lib().zero_plan_bucket(plan, k, C.byref(s), C.byref(n)), "zero_plan_bucket")
+    return s.value, n.value
+
+
+def zero_plan_segments(plan: int) -> list[tuple[int, int, int, int, int]]:
+    n = C.c_int64()
+    _check(lib().zero_plan_segments(plan, None, 0, C.byref(n)), "zero_plan_segments")
+    arr = (Segment * max(n.value, 1))()
+    _check(lib().zero_plan_segments(plan, C.cast(arr, C.c_void_p), n.value, C.byref(n)),
+           "zero_plan_segments")
+    return [(s.tensor, s.owner, s.offset_in_tensor, s.length, s.offset_in_shard)
+            for s in arr[:n.value]]
+
+
+def zero_plan_destroy(plan: int) -> None:
+    if plan:
+        lib().zero_plan_destroy(plan)
+
+
+def zero_state_bytes(psi: int, nd: int, stage: int, align_elems: int = 1) -> dict:
+    r = StateReport()
+    _check(lib().zero_state_bytes(psi, nd, stage, align_elems, C.byref(r)), "zero_state_bytes")
+    return {name: getattr(r, name) for name, _ in StateReport._fields_}
+
+
+def zero_opt_state_init(opt_state: int, stream: int = 0) -> None:
+    _check(lib().zero_opt_state_init(opt_state, stream), "zero_opt_state_init")
+
+
+def zero_workspace_bytes(plan: int, hp: HParams, args: StepArgs) -> int:
+    n = C.c_size_t()
+    _check(lib().zero_workspace_bytes(plan, C.byref(hp), C.byref(args), C.byref(n)),
+           "zero_workspace_bytes")
+    return n.value
+
+
+def zero_shard_step(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
+    _check(lib().zero_shard_step(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step")
+
+
+def zero_gather_params(plan: int, shard_ptrs, params_full: int, stream: int = 0) -> None:
+    arr = (C.c_void_p * len(shard_ptrs))(*[p if p else None for p in shard_ptrs])
+    _check(lib().zero_gather_params(plan, C.cast(arr, C.c_void_p), params_full, stream),
+           "zero_gather_params")
+
+
+def zero_cast_params(plan: int, master: int, params: int, owner_first: int, owner_count: int,
+                     stream: int = 0) -> None:
+    _check(lib().zero_cast_params(plan, master, params, owner_first, owner_count, stream),
+           "zero_cast_params")
+
+
+def zero_abi_version() -> int:
+    return lib().zero_abi_version()
+
+
+def zero_strerror(status: int) -> str:
+    return lib().zero_strerror(status).decode()
+
+
+def zero_last_error() -> str:
+    return lib().zero_last_error().decode()
+
+
+def zero_launch_count() -> int:
+    return lib().zero_launch_count()
+
+
+# ---------------------------------------------------------------------------
+# struct builders
+# ---------------------------------------------------------------------------
+
+def hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_scale=1.0,
+            max_grad_norm=0.0, average_over_nd=False, mode=ZERO_MODE_SPECULATIVE) -> HParams:
+    return HParams(lr, beta1, beta2, eps, weight_decay, loss_scale, max_grad_norm,
+                   int(average_over_nd), mode, 0)
+
+
+def step_args(*, grads: int, grad_rank_stride: int, master, exp_avg, exp_avg_sq, params: int,
+              opt_state: int, workspace: int = 0, workspace_bytes: int = 0, result: int = 0,
+              grad_layout: int = ZERO_GRADS_FULL, owner_first: int = 0, owner_count: int = 1,
+              grad_stash: int = 0, timing_events=(0, 0)) -> StepArgs:
+    """master/exp_avg/exp_avg_sq: (slot0, slot1) device addresses (slot1 may be 0)."""
+    a = StepArgs()
+    a.grads = grads
+    a.grad_rank_stride = grad_rank_stride
+    a.grad_layout = grad_layout
+    a.owner_first = owner_first
+    a.owner_count = owner_count
+    a.reserved = 0
+    for k in range(2):
+        a.master[k] = master[k] or None
+        a.exp_avg[k] = exp_avg[k] or None
+        a.exp_avg_sq[k] = exp_avg_sq[k] or None
+        a.timing_events[k] = timing_events[k] or None
+    a.params = params
+    a.grad_stash = grad_stash or None
+    a.opt_state = opt_state
+    a.result = result or None
+    a.workspace = workspace or None
+    a.workspace_bytes = workspace_bytes
+    return a
+
+
+def opt_state_from_bytes(raw: bytes) -> OptState:
+    return OptState.from_buffer_copy(raw[:C.sizeof(OptState)])
+
+
+def step_result_from_bytes(raw: bytes) -> StepResult:
+    return StepResult.from_buffer_copy(raw[:C.sizeof(StepResult)])

@@ -1,0 +1,373 @@
+// api.cpp -- C ABI entry points of libzero_shard.so that touch the device:
+// argument validation, launch planning and the per-mode kernel sequences.
+// Nothing here allocates device memory or synchronises a stream.
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "zs_internal.h"
+
+using zs::fail;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The kernel launches of one zero_shard_step call.
+struct LaunchPlan {
+    bool vec = false;                               // 16-byte vector path
+    std::vector<std::vector<zs::SegList>> buckets;  // grad-reading launches, bucket by bucket
+    std::vector<zs::SegList> whole;                 // the call's full range
+    int64_t n_partials = 0;                         // fp64 norm partials of all statistics launches
+};
+
+void push_seg(std::vector<zs::SegList>& lists, const zs::Seg& s)
+{
+    if (s.n <= 0)
+        return;
+    if (lists.empty() || lists.back().count == zs::kMaxSegs) {
+        zs::SegList l;
+        std::memset(&l, 0, sizeof l);
+        lists.push_back(l);
+    }
+    lists.back().seg[lists.back().count++] = s;
+}
+
+// Segments covering flat range [lo, hi) of the owners starting at o0.
+void segments_of(const zero_plan_s& p, int layout, int64_t stride, int32_t o0, int64_t lo,
+                 int64_t hi, std::vector<zs::SegList>& out)
+{
+    const int64_t L = p.shard_len;
+    if (lo >= hi)
+        return;
+    if (layout == ZERO_GRADS_FULL) {
+        // every array is addressed by the flat index, so owners run together
+        push_seg(out, zs::Seg{lo, stride, lo - (int64_t)o0 * L, lo, hi - lo});
+        return;
+    }
+    for (int64_t o = lo / L; o * L < hi; ++o) {
+        const int64_t i0 = (lo > o * L ? lo : o * L) - o * L;
+        const int64_t i1 = (hi < (o + 1) * L ? hi : (o + 1) * L) - o * L;
+        const int64_t j = o - o0;
+        push_seg(out, zs::Seg{j * p.nd * stride + i0, stride, j * L + i0, o * L + i0, i1 - i0});
+    }
+}
+
+bool segs_vec_ok(const std::vector<zs::SegList>& lists)
+{
+    for (const auto& l : lists)
+        for (int i = 0; i < l.count; ++i)
+            if ((l.seg[i].g_off | l.seg[i].s_off | l.seg[i].p_off | l.seg[i].g_rstride) & 7)
+                return false;
+    return true;
+}
+
+int64_t effective_stride(const zero_plan_s& p, const zero_step_args& a)
+{
+    if (a.grad_layout == ZERO_GRADS_PER_OWNER && a.grad_rank_stride == 0)
+        return p.shard_len;
+    return a.grad_rank_stride;
+}
+
+zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_step_args* a)
+{
+    if (!p || !hp || !a)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_shard_step: null plan, hparams or args");
+    if (hp->mode < ZERO_MODE_SPECULATIVE || hp->mode > ZERO_MODE_STASH)
+        return fail(ZERO_ERR_INVALID_ARG, "unknown mode %d", hp->mode);
+    if (hp->reserved != 0 || a->reserved != 0)
+        return fail(ZERO_ERR_INVALID_ARG, "reserved fields must be 0");
+    if (!(hp->loss_scale > 0.0f) || !std::isfinite(hp->loss_scale))
+        return fail(ZERO_ERR_INVALID_ARG, "loss_scale must be finite and > 0");
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay) || !std::isfinite(hp->eps) ||
+        hp->eps < 0.0f || !std::isfinite(hp->max_grad_norm))
+        return fail(ZERO_ERR_INVALID_ARG, "lr, weight_decay, eps, max_grad_norm must be finite, eps >= 0");
+    if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f))
+        return fail(ZERO_ERR_INVALID_ARG, "betas must lie in [0, 1)");
+    if (hp->average_over_nd != 0 && hp->average_over_nd != 1)
+        return fail(ZERO_ERR_INVALID_ARG, "average_over_nd must be 0 or 1");
+    if (hp->mode == ZERO_MODE_SPECULATIVE && hp->max_grad_norm > 0.0f)
+        return fail(ZERO_ERR_UNSUPPORTED, "global-norm clipping needs the norm before any update: "
+                    "use TWO_PASS or STASH mode");
+    if (a->owner_first < 0 || a->owner_count < 1 || a->owner_first > p->nd - a->owner_count)
+        return fail(ZERO_ERR_INVALID_ARG, "owner range [%d, %d + %d) outside [0, %d)",
+                    a->owner_first, a->owner_first, a->owner_count, p->nd);
+    if (a->grad_layout != ZERO_GRADS_FULL && a->grad_layout != ZERO_GRADS_PER_OWNER)
+        return fail(ZERO_ERR_INVALID_ARG, "unknown grad_layout %d", a->grad_layout);
+    const int64_t stride = effective_stride(*p, *a);
+    if (a->grad_layout == ZERO_GRADS_FULL && p->nd > 1 && stride < p->psi)
+        return fail(ZERO_ERR_INVALID_ARG, "FULL layout needs grad_rank_stride >= psi (%lld < %lld)",
+                    (long long)stride, (long long)p->psi);
+    if (a->grad_layout == ZERO_GRADS_PER_OWNER && stride < p->shard_len)
+        return fail(ZERO_ERR_INVALID_ARG, "PER_OWNER layout needs grad_rank_stride >= L (%lld < %lld)",
+                    (long long)stride, (long long)p->shard_len);
+    if (!a->grads || !a->master[0] || !a->exp_avg[0] || !a->exp_avg_sq[0] || !a->params || !a->opt_state)
+        return fail(ZERO_ERR_INVALID_ARG, "null device buffer (grads, master, exp_avg, exp_avg_sq, params, opt_state)");
+    const bool spec = hp->mode == ZERO_MODE_SPECULATIVE;
+    if (spec && (!a->master[1] || !a->exp_avg[1] || !a->exp_avg_sq[1]))
+        return fail(ZERO_ERR_INVALID_ARG, "SPECULATIVE mode needs the second state slot");
+    if (hp->mode == ZERO_MODE_STASH && !a->grad_stash)
+        return fail(ZERO_ERR_INVALID_ARG, "STASH mode needs grad_stash");
+    for (int k = 0; k < (spec ? 2 : 1); ++k)
+        if (!aligned(a->master[k], 4) || !aligned(a->exp_avg[k], 4) || !aligned(a->exp_avg_sq[k], 4))
+            return fail(ZERO_ERR_ALIGNMENT, "fp32 state buffers must be 4-byte aligned");
+    if (!aligned(a->grads, 2) || !aligned(a->params, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "fp16 buffers must be 2-byte aligned");
+    if (a->grad_stash && !aligned(a->grad_stash, 4))
+        return fail(ZERO_ERR_ALIGNMENT, "grad_stash must be 4-byte aligned");
+    if (!aligned(a->opt_state, 8) || (a->result && !aligned(a->result, 8)))
+        return fail(ZERO_ERR_ALIGNMENT, "opt_state / result must be 8-byte aligned");
+    return ZERO_OK;
+}
+
+LaunchPlan plan_launches(const zero_plan_s& p, const zero_hparams& hp, const zero_step_args& a)
+{
+    LaunchPlan lp;
+    const int64_t L = p.shard_len;
+    const int64_t stride = effective_stride(p, a);
+    const int64_t lo = (int64_t)a.owner_first * L;
+    int64_t hi = (int64_t)(a.owner_first + a.owner_count) * L;
+    if (hi > p.psi)
+        hi = p.psi;
+
+    if (p.bucket > 0) {
+        for (int64_t k = 0; k < p.n_buckets; ++k) {
+            const int64_t b0 = k * p.bucket > lo ? k * p.bucket : lo;
+            const int64_t b1 = (k + 1) * p.bucket < hi ? (k + 1) * p.bucket : hi;
+            if (b0 >= b1)
+                continue;
+            lp.buckets.emplace_back();
+            segments_of(p, a.grad_layout, stride, a.owner_first, b0, b1, lp.buckets.back());
+        }
+    } else if (lo < hi) {
+        lp.buckets.emplace_back();
+        segments_of(p, a.grad_layout, stride, a.owner_first, lo, hi, lp.buckets.back());
+    }
+    segments_of(p, a.grad_layout, stride, a.owner_first, lo, hi, lp.whole);
+    if (lp.whole.empty()) {
+        zs::SegList empty;
+        std::memset(&empty, 0, sizeof empty);
+        lp.whole.push_back(empty);
+    }
+    const bool spec = hp.mode == ZERO_MODE_SPECULATIVE;
+    bool vec = (L % 8 == 0) && (p.bucket % 8 == 0) && (stride % 8 == 0) && aligned(a.grads, 16) &&
+               aligned(a.params, 16);
+    for (int k = 0; k < (spec ? 2 : 1); ++k)
+        vec = vec && aligned(a.master[k], 16) && aligned(a.exp_avg[k], 16) && aligned(a.exp_avg_sq[k], 16);
+    if (hp.mode == ZERO_MODE_STASH)
+        vec = vec && aligned(a.grad_stash, 16);
+    vec = vec && segs_vec_ok(lp.whole);
+    for (const auto& b : lp.buckets)
+        vec = vec && segs_vec_ok(b);
+    lp.vec = vec;
+    for (const auto& b : lp.buckets)
+        for (const auto& l : b)
+            lp.n_partials += zs::stats_blocks(vec, l);
+    return lp;
+}
+
+size_t workspace_need(const zero_hparams& hp, const LaunchPlan& lp)
+{
+    if (hp.mode == ZERO_MODE_SPECULATIVE)
+        return zs::kHeaderBytes;
+    return zs::kHeaderBytes + (size_t)lp.n_partials * sizeof(double);
+}
+
+zero_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(ZERO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+} // namespace
+
+extern "C" {
+
+zero_status zero_opt_state_init(void* opt_state, void* stream)
+{
+    zs::clear_error();
+    if (!opt_state)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_opt_state_init: null opt_state");
+    if (!aligned(opt_state, 8))
+        return fail(ZERO_ERR_ALIGNMENT, "zero_opt_state_init: opt_state must be 8-byte aligned");
+    cudaError_t e = zs::launch_opt_init(static_cast<zero_opt_state*>(opt_state),
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(e, "zero_opt_state_init");
+}
+
+zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hparams* hp,
+                                 const zero_step_args* args, size_t* bytes)
+{
+    zs::clear_error();
+    if (!bytes)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_workspace_bytes: null bytes");
+    zero_status s = validate(plan, hp, args);
+    if (s != ZERO_OK)
+        return s;
+    *bytes = workspace_need(*hp, plan_launches(*plan, *hp, *args));
+    return ZERO_OK;
+}
+
+zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
+                            const zero_step_args* args, void* stream)
+{
+    zs::clear_error();
+    zero_status s = validate(plan, hp, args);
+    if (s != ZERO_OK)
+        return s;
+    const zero_plan_s& p = *plan;
+    const zero_hparams& h = *hp;
+    const zero_step_args& a = *args;
+    const LaunchPlan lp = plan_launches(p, h, a);
+    const size_t need = workspace_need(h, lp);
+    if (!a.workspace || a.workspace_bytes < need)
+        return fail(ZERO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    a.workspace ? a.workspace_bytes : (size_t)0);
+    if (!aligned(a.workspace, 256))
+        return fail(ZERO_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+
+    auto* st = static_cast<zero_opt_state*>(a.opt_state);
+    auto* res = static_cast<zero_step_result*>(a.result);
+    auto* ws = static_cast<zs::WsHeader*>(a.workspace);
+    auto* partials = reinterpret_cast<double*>(static_cast<char*>(a.workspace) + zs::kHeaderBytes);
+    cudaStream_t str = static_cast<cudaStream_t>(stream);
+    auto* ev0 = static_cast<cudaEvent_t>(a.timing_events[0]);
+    auto* ev1 = static_cast<cudaEvent_t>(a.timing_events[1]);
+
+    zs::UpdateArgs u;
+    std::memset(&u, 0, sizeof u);
+    u.grads = static_cast<const uint16_t*>(a.grads);
+    u.stash = a.grad_stash;
+    for (int k = 0; k < 2; ++k) {
+        u.master[k] = a.master[k];
+        u.exp_avg[k] = a.exp_avg[k];
+        u.exp_avg_sq[k] = a.exp_avg_sq[k];
+    }
+    u.params = static_cast<uint16_t*>(a.params);
+    u.ws = ws;
+    u.nd = p.nd;
+    double scale = (double)h.loss_scale;
+    if (h.average_over_nd)
+        scale *= (double)p.nd;
+    u.inv = (float)(1.0 / scale);
+    u.lr = h.lr;
+    u.beta1 = h.beta1;
+    u.beta2 = h.beta2;
+    u.eps = h.eps;
+    // fp32 constants, each rounded once on the host
+    u.lr_wd = h.lr * h.weight_decay;
+    u.one_minus_beta1 = 1.0f - h.beta1;
+    u.one_minus_beta2 = 1.0f - h.beta2;
+
+    cudaError_t e = zs::launch_prep(st, ws, h.beta1, h.beta2, str);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "prep launch");
+
+    if (h.mode == ZERO_MODE_SPECULATIVE) {
+        if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+            return cuda_fail(e, "timing event");
+        for (const auto& b : lp.buckets)
+            for (const auto& l : b)
+                if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, str)) != cudaSuccess)
+                    return cuda_fail(e, "update launch");
+        if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+            return cuda_fail(e, "timing event");
+        for (size_t i = 0; i < lp.whole.size(); ++i)
+            if ((e = zs::launch_commit(lp.vec, u, lp.whole[i], i == 0, st, res, str)) != cudaSuccess)
+                return cuda_fail(e, "commit launch");
+        return ZERO_OK;
+    }
+
+    // pre-pass modes: statistics bucket by bucket, finalize, in-place update
+    zs::StatsArgs sa;
+    sa.grads = u.grads;
+    sa.stash = h.mode == ZERO_MODE_STASH ? a.grad_stash : nullptr;
+    sa.ws = ws;
+    sa.nd = p.nd;
+    sa.inv = u.inv;
+    int64_t n_partials = 0;
+    for (const auto& b : lp.buckets) {
+        for (const auto& l : b) {
+            sa.partials = partials + n_partials;
+            if ((e = zs::launch_stats(lp.vec, sa, l, str)) != cudaSuccess)
+                return cuda_fail(e, "statistics launch");
+            n_partials += zs::stats_blocks(lp.vec, l);
+        }
+    }
+    if ((e = zs::launch_finalize(ws, partials, n_partials, h.max_grad_norm, st, res, str)) != cudaSuccess)
+        return cuda_fail(e, "finalize launch");
+    const int src = h.mode == ZERO_MODE_STASH ? zs::kSrcStash : zs::kSrcGradsInPlace;
+    if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+        return cuda_fail(e, "timing event");
+    for (const auto& l : lp.whole)
+        if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, str)) != cudaSuccess)
+            return cuda_fail(e, "update launch");
+    if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+        return cuda_fail(e, "timing event");
+    return ZERO_OK;
+}
+
+zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard_ptrs,
+                               void* params_full, void* stream)
+{
+    zs::clear_error();
+    if (!plan || !shard_ptrs || !params_full)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_params: null argument");
+    const zero_plan_s& p = *plan;
+    if (!aligned(params_full, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "zero_gather_params: params_full must be 2-byte aligned");
+    std::vector<zs::GatherEntry> entries;
+    bool vec = (p.shard_len % 8 == 0) && aligned(params_full, 16);
+    for (int32_t r = 0; r < p.nd; ++r) {
+        if (!shard_ptrs[r])
+            continue;
+        if (!aligned(shard_ptrs[r], 2))
+            return fail(ZERO_ERR_ALIGNMENT, "zero_gather_params: shard %d must be 2-byte aligned", r);
+        const int64_t start = (int64_t)r * p.shard_len;
+        int64_t n = p.psi - start;
+        n = n < 0 ? 0 : (n > p.shard_len ? p.shard_len : n);
+        if (n == 0)
+            continue;
+        vec = vec && aligned(shard_ptrs[r], 16);
+        entries.push_back({static_cast<const uint16_t*>(shard_ptrs[r]), start, n});
+    }
+    cudaStream_t str = static_cast<cudaStream_t>(stream);
+    for (size_t i = 0; i < entries.size(); i += zs::kMaxSegs) {
+        zs::GatherList g;
+        std::memset(&g, 0, sizeof g);
+        for (size_t k = i; k < entries.size() && g.count < zs::kMaxSegs; ++k)
+            g.e[g.count++] = entries[k];
+        cudaError_t e = zs::launch_gather(vec, static_cast<uint16_t*>(params_full), g, str);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "gather launch");
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,
+                             int32_t owner_first, int32_t owner_count, void* stream)
+{
+    zs::clear_error();
+    if (!plan || !master || !params)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_cast_params: null argument");
+    const zero_plan_s& p = *plan;
+    if (owner_first < 0 || owner_count < 1 || owner_first > p.nd - owner_count)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_cast_params: owner range outside the plan");
+    if (!aligned(master, 4) || !aligned(params, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "zero_cast_params: misaligned buffer");
+    const int64_t lo = (int64_t)owner_first * p.shard_len;
+    int64_t hi = (int64_t)(owner_first + owner_count) * p.shard_len;
+    hi = hi > p.psi ? p.psi : hi;
+    std::vector<zs::SegList> lists;
+    segments_of(p, ZERO_GRADS_FULL, 0, owner_first, lo, hi, lists);
+    const bool vec = (p.shard_len % 8 == 0) && aligned(master, 16) && aligned(params, 16) &&
+                     segs_vec_ok(lists);
+    for (const auto& l : lists) {
+        cudaError_t e = zs::launch_cast(vec, master, static_cast<uint16_t*>(params), l,
+                                        static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cast launch");
+    }
+    return ZERO_OK;
+}
+
+} // extern "C"

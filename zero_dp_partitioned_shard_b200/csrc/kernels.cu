@@ -1,0 +1,695 @@
+// kernels.cu -- sm_100a kernels of libzero_shard.so.
+//
+// The step is HBM-bound streaming work (about 20 fp32 operations, one square
+// root and three divisions per parameter against 2*Nd + 26 bytes), so it uses
+// no tensor cores.  Design points for B200:
+//   * one thread owns 8 consecutive parameters per iteration: every access is
+//     a 16-byte vector (fp16 x8 or fp32 x4) and a warp touches 512 contiguous
+//     bytes of each stream; loads bypass L1 and are marked evict-first, since
+//     every byte is read exactly once;
+//   * the Nd rank contributions of a chunk are loaded in groups of 8 before
+//     any is added, so up to 8 * 16 B of gradient plus 96 B of optimizer state
+//     are in flight per thread; the adds then run in rank order;
+//   * persistent grid-stride launches sized to (SM count x resident blocks);
+//   * the overflow flag is a warp vote followed by one atomicOr per warp that
+//     saw a non-finite value; the fp64 norm partials are reduced per block in a
+//     fixed shuffle pattern and summed in a fixed order by a one-block kernel,
+//     so results are bit-reproducible for a given launch geometry.
+// No kernel waits on another block, a flag or a peer: ordering between the
+// kernels of a step is plain stream order.
+//
+// Arithmetic per parameter (ZeRO leaves the optimizer's maths unchanged; the
+// pages name Adam with fp32 master, momentum and variance -- "ZeRO memory
+// optimization: training large models", trishampatil.com, "The Real Problem"
+// -- and the equations are the textbook Adam/AdamW of Kingma & Ba 2015, Alg. 1
+// and Loshchilov & Hutter 2019): every fp32 operation is an explicitly rounded
+// intrinsic (no contraction into FMA), division and square root are the
+// IEEE-rounded __fdiv_rn / __fsqrt_rn, and the fp16 cast is round-to-nearest-
+// even with subnormals kept.
+#include <cuda_fp16.h>
+
+#include <map>
+#include <mutex>
+#include <unordered_map>
+#include <utility>
+
+#include "zs_internal.h"
+
+namespace zs {
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+
+struct AdamK {
+    float beta1, beta2, omb1, omb2, lr, lr_wd, eps, bc1, bc2, clip;
+};
+
+// m = b1*m + (1-b1)*g; v = b2*v + (1-b2)*g^2;
+// p = (p - lr_wd*p) - lr * ((m/bc1) / (sqrt(v/bc2) + eps))
+__device__ __forceinline__ void adam_update(float g, float& p, float& m, float& v, const AdamK& k)
+{
+    const float m_new = __fadd_rn(__fmul_rn(k.beta1, m), __fmul_rn(k.omb1, g));
+    const float v_new = __fadd_rn(__fmul_rn(k.beta2, v), __fmul_rn(k.omb2, __fmul_rn(g, g)));
+    const float m_hat = __fdiv_rn(m_new, k.bc1);
+    const float v_hat = __fdiv_rn(v_new, k.bc2);
+    const float denom = __fadd_rn(__fsqrt_rn(v_hat), k.eps);
+    const float step = __fmul_rn(k.lr, __fdiv_rn(m_hat, denom));
+    p = __fsub_rn(__fsub_rn(p, __fmul_rn(k.lr_wd, p)), step);
+    m = m_new;
+    v = v_new;
+}
+
+__device__ __forceinline__ void unpack_h8(const uint4& x, float f[8])
+{
+    const __half2* h = reinterpret_cast<const __half2*>(&x);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float2 t = __half22float2(h[q]);
+        f[2 * q] = t.x;
+        f[2 * q + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ uint4 pack_h8(const float f[8])
+{
+    uint4 x;
+    __half2* h = reinterpret_cast<__half2*>(&x);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        h[q] = __floats2half2_rn(f[2 * q], f[2 * q + 1]);
+    return x;
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p)
+{
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void ld_f8(const float* p, float f[8])
+{
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+__device__ __forceinline__ void st_f8(float* p, const float f[8])
+{
+    __stcs(reinterpret_cast<float4*>(p), make_float4(f[0], f[1], f[2], f[3]));
+    __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(f[4], f[5], f[6], f[7]));
+}
+
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+
+// Rank-order sum of the Nd contributions of 8 consecutive parameters: the
+// loads of each group of 8 ranks are issued together, then added in order.
+__device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, int nd, float s[8])
+{
+    {
+        uint4 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (u < nd)
+                x[u] = ld_stream(g + u * rstride);
+        unpack_h8(x[0], s);
+#pragma unroll
+        for (int u = 1; u < 8; ++u) {
+            if (u < nd) {
+                float f[8];
+                unpack_h8(x[u], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    s[q] = __fadd_rn(s[q], f[q]);
+            }
+        }
+    }
+    for (int r = 8; r < nd; r += 8) {
+        uint4 x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (r + u < nd)
+                x[u] = ld_stream(g + (int64_t)(r + u) * rstride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (r + u < nd) {
+                float f[8];
+                unpack_h8(x[u], f);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    s[q] = __fadd_rn(s[q], f[q]);
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float rank_sum1(const uint16_t* g, int64_t rstride, int nd)
+{
+    float s = h2f(g[0]);
+    for (int r = 1; r < nd; ++r)
+        s = __fadd_rn(s, h2f(g[(int64_t)r * rstride]));
+    return s;
+}
+
+__device__ __forceinline__ void flag_nonfinite(bool bad, unsigned int* flag)
+{
+    // every lane of the warp reaches this point (grid-stride loops only)
+    const unsigned int any = __ballot_sync(0xffffffffu, bad);
+    if (any && (threadIdx.x & 31) == 0)
+        atomicOr(flag, 1u);
+}
+
+__device__ __forceinline__ AdamK load_consts(const UpdateArgs& a, const WsHeader* ws, bool clip)
+{
+    AdamK k;
+    k.beta1 = a.beta1;
+    k.beta2 = a.beta2;
+    k.omb1 = a.one_minus_beta1;
+    k.omb2 = a.one_minus_beta2;
+    k.lr = a.lr;
+    k.lr_wd = a.lr_wd;
+    k.eps = a.eps;
+    k.bc1 = ws->bc1;
+    k.bc2 = ws->bc2;
+    k.clip = clip ? ws->clip : 1.0f;
+    return k;
+}
+
+// ---------------------------------------------------------------------------
+// K0: optimizer-state init and per-step prep (one thread)
+// ---------------------------------------------------------------------------
+
+__global__ void zs_opt_init_kernel(zero_opt_state* st)
+{
+    st->t = 0;
+    st->beta1_pow = 1.0;
+    st->beta2_pow = 1.0;
+    st->skipped = 0;
+    st->cur = 0;
+    st->reserved = 0;
+}
+
+// Bias corrections of the step about to be applied, from the fp64 running
+// products beta^t: bc = (fp32)(1 - beta^(t+1)).
+__global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2)
+{
+    const double b1 = __dmul_rn(st->beta1_pow, (double)beta1);
+    const double b2 = __dmul_rn(st->beta2_pow, (double)beta2);
+    ws->overflow = 0u;
+    ws->skip = 0;
+    ws->cur = st->cur & 1;
+    ws->bc1 = __double2float_rn(__dsub_rn(1.0, b1));
+    ws->bc2 = __double2float_rn(__dsub_rn(1.0, b2));
+    ws->clip = 1.0f;
+    ws->b1p_next = b1;
+    ws->b2p_next = b2;
+    ws->sumsq = 0.0;
+    ws->norm = __longlong_as_double(0x7ff8000000000000LL);
+    ws->t_next = st->t + 1;
+}
+
+// ---------------------------------------------------------------------------
+// K1: fused reduce + unscale (+ overflow) + clip + Adam + fp16 cast
+// ---------------------------------------------------------------------------
+
+template <int SRC, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
+{
+    constexpr bool kSpec = SRC == kSrcGradsSpeculative;
+    const WsHeader* ws = a.ws;
+    if (!kSpec && ws->skip)
+        return; // uniform across the grid: the whole step is skipped
+    const int cur = kSpec ? ws->cur : 0;
+    const int nxt = kSpec ? cur ^ 1 : 0;
+    const AdamK k = load_consts(a, ws, !kSpec);
+    // slot selection by value: indexing the parameter arrays with a runtime
+    // index would force a local-memory copy of the whole argument struct
+    const float* __restrict__ p_in = cur ? a.master[1] : a.master[0];
+    const float* __restrict__ m_in = cur ? a.exp_avg[1] : a.exp_avg[0];
+    const float* __restrict__ v_in = cur ? a.exp_avg_sq[1] : a.exp_avg_sq[0];
+    float* p_out = nxt ? a.master[1] : a.master[0];
+    float* m_out = nxt ? a.exp_avg[1] : a.exp_avg[0];
+    float* v_out = nxt ? a.exp_avg_sq[1] : a.exp_avg_sq[0];
+
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    bool bad = false;
+
+    for (int si = 0; si < segs.count; ++si) {
+        const Seg& sg = segs.seg[si];
+        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
+        for (int64_t c = tid; c < n_vec; c += nthr) {
+            const int64_t e = c << 3;
+            const int64_t so = sg.s_off + e;
+            float p[8], m[8], v[8], g[8];
+            ld_f8(p_in + so, p);
+            ld_f8(m_in + so, m);
+            ld_f8(v_in + so, v);
+            if (SRC == kSrcStash) {
+                ld_f8(a.stash + so, g);
+            } else {
+                rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    g[q] = __fmul_rn(g[q], a.inv);
+            }
+            if (kSpec) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    bad |= !isfinite(g[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                adam_update(__fmul_rn(g[q], k.clip), p[q], m[q], v[q], k);
+            st_f8(p_out + so, p);
+            st_f8(m_out + so, m);
+            st_f8(v_out + so, v);
+            __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8(p));
+        }
+        // scalar elements: everything (VEC = false) or the < 8 tail
+        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr) {
+            const int64_t so = sg.s_off + e;
+            float g;
+            if (SRC == kSrcStash)
+                g = a.stash[so];
+            else
+                g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
+            if (kSpec)
+                bad |= !isfinite(g);
+            float p = p_in[so], m = m_in[so], v = v_in[so];
+            adam_update(__fmul_rn(g, k.clip), p, m, v, k);
+            p_out[so] = p;
+            m_out[so] = m;
+            v_out[so] = v;
+            a.params[sg.p_off + e] = f2h(p);
+        }
+    }
+    if (kSpec)
+        flag_nonfinite(bad, &a.ws->overflow);
+}
+
+// ---------------------------------------------------------------------------
+// K2: statistics pre-pass -- overflow flag, fp64 sum of squares per block,
+//     optionally the fp32 reduced gradient (stash)
+// ---------------------------------------------------------------------------
+
+template <bool VEC, bool STASH>
+__global__ void __launch_bounds__(kThreads)
+zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
+{
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    double acc = 0.0;
+    bool bad = false;
+    for (int si = 0; si < segs.count; ++si) {
+        const Seg& sg = segs.seg[si];
+        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
+        for (int64_t c = tid; c < n_vec; c += nthr) {
+            const int64_t e = c << 3;
+            float g[8];
+            rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                g[q] = __fmul_rn(g[q], a.inv);
+                bad |= !isfinite(g[q]);
+                const double d = (double)g[q];
+                acc = __dadd_rn(acc, __dmul_rn(d, d));
+            }
+            if (STASH)
+                st_f8(a.stash + sg.s_off + e, g);
+        }
+        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr) {
+            const float g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
+            bad |= !isfinite(g);
+            const double d = (double)g;
+            acc = __dadd_rn(acc, __dmul_rn(d, d));
+            if (STASH)
+                a.stash[sg.s_off + e] = g;
+        }
+    }
+    flag_nonfinite(bad, &a.ws->overflow);
+
+    // fixed-pattern block reduction of the fp64 partial sums
+    __shared__ double warp_sum[kThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+    if ((threadIdx.x & 31) == 0)
+        warp_sum[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        double w = threadIdx.x < kThreads / 32 ? warp_sum[threadIdx.x] : 0.0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            w = __dadd_rn(w, __shfl_down_sync(0xffffffffu, w, off));
+        if (threadIdx.x == 0)
+            a.partials[blockIdx.x] = w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K3: finalize (one block) -- norm, clip coefficient, skip, bookkeeping
+// ---------------------------------------------------------------------------
+
+constexpr int kFinalizeThreads = 1024;
+
+__global__ void __launch_bounds__(kFinalizeThreads)
+zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_norm,
+                   zero_opt_state* st, zero_step_result* res)
+{
+    double acc = 0.0;
+    for (int64_t i = threadIdx.x; i < n; i += kFinalizeThreads)
+        acc = __dadd_rn(acc, partials[i]);
+    __shared__ double warp_sum[kFinalizeThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+    if ((threadIdx.x & 31) == 0)
+        warp_sum[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x >= 32)
+        return;
+    double w = warp_sum[threadIdx.x];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        w = __dadd_rn(w, __shfl_down_sync(0xffffffffu, w, off));
+    if (threadIdx.x != 0)
+        return;
+    const bool skip = ws->overflow != 0u;
+    const double norm = __dsqrt_rn(w);
+    float clip = 1.0f;
+    if (!skip && max_norm > 0.0f && norm > (double)max_norm)
+        clip = __double2float_rn(__ddiv_rn((double)max_norm, norm));
+    ws->skip = skip ? 1 : 0;
+    ws->clip = clip;
+    ws->sumsq = w;
+    ws->norm = norm;
+    if (!skip) {
+        st->t = ws->t_next;
+        st->beta1_pow = ws->b1p_next;
+        st->beta2_pow = ws->b2p_next;
+    } else {
+        st->skipped += 1;
+    }
+    if (res) {
+        res->grad_norm = skip ? __longlong_as_double(0x7ff8000000000000LL) : norm;
+        res->t = st->t;
+        res->skipped = st->skipped;
+        res->clip_coef = clip;
+        res->overflow = skip ? 1 : 0;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// K5: speculative commit -- flip the live slot, or on overflow re-cast the
+//     fp16 parameters from the unchanged live master; also zero_cast_params
+// ---------------------------------------------------------------------------
+
+template <bool VEC>
+__device__ __forceinline__ void cast_segments(const float* master, uint16_t* params, const SegList& segs)
+{
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    for (int si = 0; si < segs.count; ++si) {
+        const Seg& sg = segs.seg[si];
+        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
+        for (int64_t c = tid; c < n_vec; c += nthr) {
+            const int64_t e = c << 3;
+            float p[8];
+            ld_f8(master + sg.s_off + e, p);
+            __stcs(reinterpret_cast<uint4*>(params + sg.p_off + e), pack_h8(p));
+        }
+        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr)
+            params[sg.p_off + e] = f2h(master[sg.s_off + e]);
+    }
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads)
+zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int bookkeeping,
+                 zero_opt_state* st, zero_step_result* res)
+{
+    const WsHeader* ws = a.ws;
+    const bool over = ws->overflow != 0u;
+    const int cur = ws->cur;
+    if (bookkeeping && blockIdx.x == 0 && threadIdx.x == 0) {
+        if (!over) {
+            st->t = ws->t_next;
+            st->beta1_pow = ws->b1p_next;
+            st->beta2_pow = ws->b2p_next;
+            st->cur = cur ^ 1;
+        } else {
+            st->skipped += 1;
+        }
+        if (res) {
+            res->grad_norm = __longlong_as_double(0x7ff8000000000000LL);
+            res->t = st->t;
+            res->skipped = st->skipped;
+            res->clip_coef = 1.0f;
+            res->overflow = over ? 1 : 0;
+        }
+    }
+    if (!over)
+        return;
+    cast_segments<VEC>(cur ? a.master[1] : a.master[0], a.params, segs);
+}
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads)
+zs_cast_kernel(const float* master, uint16_t* params, const __grid_constant__ SegList segs)
+{
+    cast_segments<VEC>(master, params, segs);
+}
+
+// ---------------------------------------------------------------------------
+// K4: gather-assembly of fp16 parameter shards into the full buffer
+// ---------------------------------------------------------------------------
+
+template <bool VEC>
+__global__ void __launch_bounds__(kThreads)
+zs_gather_kernel(uint16_t* dst, const __grid_constant__ GatherList g)
+{
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    for (int k = 0; k < g.count; ++k) {
+        const GatherEntry& ge = g.e[k];
+        uint16_t* out = dst + ge.dst_off;
+        const int64_t n_vec = VEC ? (ge.n >> 3) : 0;
+        for (int64_t c = tid; c < n_vec; c += nthr)
+            __stcs(reinterpret_cast<uint4*>(out) + c, ld_stream(ge.src + (c << 3)));
+        for (int64_t e = (n_vec << 3) + tid; e < ge.n; e += nthr)
+            out[e] = ge.src[e];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launch geometry
+// ---------------------------------------------------------------------------
+
+struct DevInfo {
+    int sms = 0;
+};
+
+static std::mutex g_mu;
+static std::unordered_map<int, DevInfo> g_dev;
+static std::map<std::pair<const void*, int>, int> g_occ; // (kernel, device) -> blocks per SM
+
+static cudaError_t device_sms(int* sms)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        DevInfo d;
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return e;
+        it = g_dev.emplace(dev, d).first;
+    }
+    *sms = it->second.sms;
+    return cudaSuccess;
+}
+
+// Persistent grid: SM count x resident blocks, but no more blocks than work.
+template <typename K>
+static cudaError_t grid_for(K kernel, int64_t work_threads, int cap, int* blocks)
+{
+    int sms = 0;
+    cudaError_t e = device_sms(&sms);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess)
+        return e;
+    const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+    int occ = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_occ.find(key);
+        if (it != g_occ.end())
+            occ = it->second;
+    }
+    if (occ == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0);
+        if (e != cudaSuccess)
+            return e;
+        if (occ < 1)
+            occ = 1;
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_occ[key] = occ;
+    }
+    int64_t want = (work_threads + kThreads - 1) / kThreads;
+    int64_t full = (int64_t)sms * occ;
+    if (cap > 0 && full > cap)
+        full = cap;
+    *blocks = (int)(want < 1 ? 1 : (want < full ? want : full));
+    return cudaSuccess;
+}
+
+static int64_t seg_work(const SegList& s, bool vec)
+{
+    int64_t w = 0;
+    for (int i = 0; i < s.count; ++i) {
+        const int64_t t = vec ? (s.seg[i].n + 7) >> 3 : s.seg[i].n;
+        w = t > w ? t : w;
+    }
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+cudaError_t launch_opt_init(zero_opt_state* st, cudaStream_t s)
+{
+    zs_opt_init_kernel<<<1, 1, 0, s>>>(st);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2,
+                        cudaStream_t s)
+{
+    zs_prep_kernel<<<1, 1, 0, s>>>(st, ws, beta1, beta2);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int SRC, bool VEC>
+static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+{
+    int blocks = 0;
+    cudaError_t e = grid_for(zs_update_kernel<SRC, VEC>, seg_work(segs, VEC), 0, &blocks);
+    if (e != cudaSuccess)
+        return e;
+    zs_update_kernel<SRC, VEC><<<blocks, kThreads, 0, s>>>(a, segs);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+{
+    switch (src) {
+    case kSrcGradsSpeculative:
+        return vec ? launch_update_t<kSrcGradsSpeculative, true>(a, segs, s)
+                   : launch_update_t<kSrcGradsSpeculative, false>(a, segs, s);
+    case kSrcGradsInPlace:
+        return vec ? launch_update_t<kSrcGradsInPlace, true>(a, segs, s)
+                   : launch_update_t<kSrcGradsInPlace, false>(a, segs, s);
+    default:
+        return vec ? launch_update_t<kSrcStash, true>(a, segs, s)
+                   : launch_update_t<kSrcStash, false>(a, segs, s);
+    }
+}
+
+int stats_blocks(bool vec, const SegList& segs)
+{
+    // a function of the work alone (not of the device), so the workspace size
+    // and the fp64 summation order are the same on every GPU
+    const int64_t want = (seg_work(segs, vec) + kThreads - 1) / kThreads;
+    return (int)(want < 1 ? 1 : (want > kStatsMaxBlocks ? kStatsMaxBlocks : want));
+}
+
+template <bool VEC, bool STASH>
+static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, cudaStream_t s)
+{
+    zs_stats_kernel<VEC, STASH><<<stats_blocks(VEC, segs), kThreads, 0, s>>>(a, segs);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
+{
+    const bool stash = a.stash != nullptr;
+    if (vec)
+        return stash ? launch_stats_t<true, true>(a, segs, s) : launch_stats_t<true, false>(a, segs, s);
+    return stash ? launch_stats_t<false, true>(a, segs, s) : launch_stats_t<false, false>(a, segs, s);
+}
+
+cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, float max_norm,
+                            zero_opt_state* st, zero_step_result* res, cudaStream_t s)
+{
+    zs_finalize_kernel<<<1, kFinalizeThreads, 0, s>>>(ws, partials, n, max_norm, st, res);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
+                          zero_opt_state* st, zero_step_result* res, cudaStream_t s)
+{
+    int blocks = 0;
+    cudaError_t e = vec ? grid_for(zs_commit_kernel<true>, seg_work(segs, true), 0, &blocks)
+                        : grid_for(zs_commit_kernel<false>, seg_work(segs, false), 0, &blocks);
+    if (e != cudaSuccess)
+        return e;
+    if (vec)
+        zs_commit_kernel<true><<<blocks, kThreads, 0, s>>>(a, segs, bookkeeping ? 1 : 0, st, res);
+    else
+        zs_commit_kernel<false><<<blocks, kThreads, 0, s>>>(a, segs, bookkeeping ? 1 : 0, st, res);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
+                        cudaStream_t s)
+{
+    int blocks = 0;
+    cudaError_t e = vec ? grid_for(zs_cast_kernel<true>, seg_work(segs, true), 0, &blocks)
+                        : grid_for(zs_cast_kernel<false>, seg_work(segs, false), 0, &blocks);
+    if (e != cudaSuccess)
+        return e;
+    if (vec)
+        zs_cast_kernel<true><<<blocks, kThreads, 0, s>>>(master, params, segs);
+    else
+        zs_cast_kernel<false><<<blocks, kThreads, 0, s>>>(master, params, segs);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(bool vec, uint16_t* dst, const GatherList& g, cudaStream_t s)
+{
+    int64_t w = 0;
+    for (int i = 0; i < g.count; ++i) {
+        const int64_t t = vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
+        w = t > w ? t : w;
+    }
+    int blocks = 0;
+    cudaError_t e = vec ? grid_for(zs_gather_kernel<true>, w, 0, &blocks)
+                        : grid_for(zs_gather_kernel<false>, w, 0, &blocks);
+    if (e != cudaSuccess)
+        return e;
+    if (vec)
+        zs_gather_kernel<true><<<blocks, kThreads, 0, s>>>(dst, g);
+    else
+        zs_gather_kernel<false><<<blocks, kThreads, 0, s>>>(dst, g);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+} // namespace zs

@@ -1,0 +1,130 @@
+// zs_internal.h -- types shared by the host API (api.cpp, plan.cpp) and the
+// kernels (kernels.cu) of libzero_shard.so.  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "zero_shard.h"
+
+struct zero_plan_s {
+    int64_t psi = 0;
+    int64_t shard_len = 0; // L
+    int64_t psi_pad = 0;   // Nd * L
+    int64_t align = 1;     // A
+    int64_t bucket = 0;    // B (0: one bucket)
+    int64_t n_buckets = 1;
+    int32_t nd = 1;
+    int32_t stage = 0;
+    std::vector<zero_segment> segments; // tensor -> owner pieces (optional)
+};
+
+namespace zs {
+
+// ---- error reporting (plan.cpp) ---------------------------------------------
+zero_status fail(zero_status s, const char* fmt, ...);
+void clear_error();
+void count_launches(uint64_t n);
+
+// ---- launch geometry ------------------------------------------------------------
+constexpr int kThreads = 256;          // threads per block of the streaming kernels
+constexpr int kMaxSegs = 64;           // segments per launch (kernel parameter table)
+constexpr int kStatsMaxBlocks = 2048;  // fp64 norm partials per statistics launch
+constexpr size_t kHeaderBytes = 256;   // workspace header, before the partials
+
+// A contiguous run of n elements processed by one kernel launch.  Element e
+// (0 <= e < n) reads rank r's fp16 contribution at grads[g_off + r*g_rstride + e],
+// the fp32 state at [s_off + e] and writes the fp16 parameter at params[p_off + e].
+struct Seg {
+    int64_t g_off;
+    int64_t g_rstride;
+    int64_t s_off;
+    int64_t p_off;
+    int64_t n;
+};
+
+struct SegList {
+    int32_t count;
+    int32_t pad;
+    Seg seg[kMaxSegs];
+};
+
+// Per-step scalars in the device workspace.  Written by the prep kernel from
+// the optimizer state, completed by the finalize / commit kernels.
+struct WsHeader {
+    unsigned int overflow; // any non-finite reduced gradient seen (atomicOr)
+    int32_t skip;          // pre-pass modes: the step is skipped
+    int32_t cur;           // live ping-pong slot at the start of the step
+    float bc1, bc2;        // bias corrections of the step being applied
+    float clip;            // clip coefficient applied by the update
+    int32_t pad0;
+    double b1p_next, b2p_next;
+    double sumsq, norm;
+    int64_t t_next;
+};
+static_assert(sizeof(WsHeader) <= kHeaderBytes, "workspace header too large");
+
+// Source of the reduced gradient in the update kernel.
+enum UpdateSrc : int {
+    kSrcGradsSpeculative = 0, // fused reduce, overflow flag, ping-pong state
+    kSrcGradsInPlace = 1,     // TWO_PASS: re-reduce; skip decided beforehand
+    kSrcStash = 2,            // STASH: read the fp32 reduced gradient
+};
+
+struct UpdateArgs {
+    const uint16_t* grads;
+    const float* stash;
+    float* master[2];
+    float* exp_avg[2];
+    float* exp_avg_sq[2];
+    uint16_t* params;
+    WsHeader* ws;
+    int32_t nd;
+    float inv;                         // fp32 1/S (or 1/(S*Nd))
+    float lr, beta1, beta2, eps, lr_wd;
+    float one_minus_beta1, one_minus_beta2;
+};
+
+struct StatsArgs {
+    const uint16_t* grads;
+    float* stash; // nullptr unless STASH
+    WsHeader* ws;
+    double* partials;
+    int32_t nd;
+    float inv;
+};
+
+struct GatherEntry {
+    const uint16_t* src;
+    int64_t dst_off;
+    int64_t n;
+};
+
+struct GatherList {
+    int32_t count;
+    int32_t pad;
+    GatherEntry e[kMaxSegs];
+};
+
+// ---- launchers (kernels.cu); each returns the launch's cudaError_t ----------
+cudaError_t launch_opt_init(zero_opt_state* st, cudaStream_t s);
+cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2,
+                        cudaStream_t s);
+cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs,
+                          cudaStream_t s);
+// blocks (= fp64 partials written) of one statistics launch over segs
+int stats_blocks(bool vec, const SegList& segs);
+cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s);
+cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n_partials,
+                            float max_grad_norm, zero_opt_state* st, zero_step_result* res,
+                            cudaStream_t s);
+cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
+                          zero_opt_state* st, zero_step_result* res, cudaStream_t s);
+cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
+                        cudaStream_t s);
+cudaError_t launch_gather(bool vec, uint16_t* dst, const GatherList& g, cudaStream_t s);
+
+} // namespace zs
