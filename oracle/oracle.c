@@ -38,9 +38,10 @@
  *   - Unscaling multiplies by the fp32 reciprocal of the loss scale.
  *   - Overflow: any non-finite reduced, unscaled gradient element skips the
  *     whole step; no state, no parameter and no step counter changes.
- *   - Clipping: global L2 norm over all real elements (pads excluded),
- *     accumulated in fp64 left to right; coefficient max/norm only when the
- *     norm exceeds max.
+ *   - Clipping: global L2 norm over all real elements (pads excluded); the
+ *     sum of squares is the exact one to within a few fp64 ulp (Neumaier's
+ *     compensated summation, 1974, of the exact fp64 squares of the fp32
+ *     gradient); coefficient max/norm only when the norm exceeds max.
  *   - Bias corrections: running products beta^t in fp64, 1 - beta^t rounded
  *     to fp32.
  *   - Padding: equal shards of L = ceil(Psi/(Nd*A))*A elements.
@@ -410,6 +411,23 @@ typedef struct {
     float lr, lr_wd, eps, bc1, bc2, clip;
 } adam_consts;
 
+/* Compensated running sum (Neumaier 1974): s holds the sum, c the lost
+ * low-order part; s + c is the total to within about one ulp, whatever the
+ * number of terms. */
+typedef struct {
+    double s, c;
+} comp_sum;
+
+static void comp_add(comp_sum* a, double t)
+{
+    double y = a->s + t;
+    if (fabs(a->s) >= fabs(t))
+        a->c += (a->s - y) + t;
+    else
+        a->c += (t - y) + a->s;
+    a->s = y;
+}
+
 /* Unscale factor: fp32 reciprocal of S (times 1/Nd when averaging). */
 static float unscale_factor(const oracle_hparams* hp, int32_t nd)
 {
@@ -532,10 +550,12 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
         return 0;
     }
 
-    /* 3. global norm, fp64, left to right; clip coefficient */
-    double sumsq = 0.0;
+    /* 3. global L2 norm: the exact fp64 squares, summed with compensation;
+     * clip coefficient */
+    comp_sum acc = {0.0, 0.0};
     for (int64_t i = 0; i < psi; ++i)
-        sumsq += (double)g[i] * (double)g[i];
+        comp_add(&acc, (double)g[i] * (double)g[i]);
+    double sumsq = acc.s + acc.c;
     double norm = sqrt(sumsq);
     float clip = 1.0f;
     if (hp->max_grad_norm > 0.0f && norm > (double)hp->max_grad_norm)
@@ -570,19 +590,20 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
     return 0;
 }
 
-/* Sum of squares of the unscaled reduced gradient over n elements, fp64 left
- * to right, continuing from acc (lets a caller stream a large problem through
- * in order).  Returns the new accumulator; *nonfinite is set to 1 if any
- * reduced element is non-finite. */
+/* Sum of squares of the unscaled reduced gradient over n elements (the same
+ * compensated fp64 sum as oracle_step), added to acc.  Lets a caller stream a
+ * large problem through in pieces.  *nonfinite is set to 1 if any reduced
+ * element is non-finite. */
 double oracle_grad_sumsq(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t n,
                          const oracle_hparams* hp, double acc, int32_t* nonfinite)
 {
     const float inv = unscale_factor(hp, nd);
+    comp_sum a = {acc, 0.0};
     for (int64_t i = 0; i < n; ++i) {
         float g = rank_sum(G, rank_stride, nd, i) * inv;
         if (!isfinite(g))
             *nonfinite = 1;
-        acc += (double)g * (double)g;
+        comp_add(&a, (double)g * (double)g);
     }
-    return acc;
+    return a.s + a.c;
 }

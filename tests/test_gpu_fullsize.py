@@ -202,13 +202,19 @@ def test_7p5b_gather_assembly_sampled_windows():
 def _streamed_oracle_norm(bn, hp, chunk=1 << 24):
     """Oracle fp64 sum of squares over all owned elements, chunk by chunk from
     the device bytes (chunks summed in order; within a chunk left to right)."""
-    jobs = []
-    for s in range(0, bn.owned, chunk):
+    starts = list(range(0, bn.owned, chunk))
+    workers = oracle.host_threads()
+    parts = []
+
+    def load(s):
         e = min(bn.owned, s + chunk)
         G = torch.stack([bn.grads[r * bn.stride + s:r * bn.stride + e] for r in range(bn.nd)])
-        jobs.append(G.view(torch.int16).cpu().numpy().view(np.uint16))
-    with cf.ThreadPoolExecutor(max_workers=oracle.host_threads()) as ex:
-        parts = list(ex.map(lambda G: oracle.grad_sumsq(G, hp), jobs))
+        return G.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        for w in range(0, len(starts), workers):   # bounded host memory: one wave at a time
+            wave = [load(s) for s in starts[w:w + workers]]
+            parts += list(ex.map(lambda G: oracle.grad_sumsq(G, hp), wave))
     total = 0.0
     bad = False
     for s, b in parts:

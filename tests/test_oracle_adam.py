@@ -147,6 +147,23 @@ def test_norm_of_constant_contributions(nd, psi, S, c):
     assert s == infos[0]["sumsq"] and not bad
 
 
+def test_norm_is_the_exact_sum_of_squares():
+    """The oracle's sum of squares equals the exactly rounded sum (math.fsum)
+    of the exact fp64 squares of the fp32 reduced gradient, to 2 ulp, even
+    over many terms of mixed magnitude, where a left-to-right fp64 sum drifts."""
+    nd, n, S = 4, 1 << 20, 1024.0
+    G = synth.grads_f16(nd, n, seed=31, std=1e-3, scale=S)
+    G[:, ::977] = np.float16(1000.0).view(np.uint16)   # a few large terms
+    g = oracle.all_reduce(G, n) * np.float32(1.0 / S)    # fp32, as the step unscales
+    exact = math.fsum((g.astype(np.float64) ** 2).tolist())
+    hp = oracle.HP(loss_scale=S)
+    s, bad = oracle.grad_sumsq(G, hp)
+    assert not bad and abs(s - exact) <= 2 * math.ulp(exact)
+    _, _, _, _, _, infos = _run(G, np.zeros(n, F32), hp, 1)
+    assert abs(infos[0]["sumsq"] - exact) <= 2 * math.ulp(exact)
+    assert infos[0]["grad_norm"] == math.sqrt(infos[0]["sumsq"])
+
+
 def test_average_over_nd_divides_by_nd():
     nd, n, S = 8, 64, 1024.0
     G, g = _const_grads(np.full(n, 2.0 ** -8), nd, S)
