@@ -275,6 +275,40 @@ ZERO_API zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hp
 ZERO_API zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
                             const zero_step_args* args, void* stream);
 
+/* Size of the device scratch array that zero_shard_step_static_scratch uses
+ * (1 MiB on every GPU that loads the library, kept until the process exits). */
+#define ZERO_STATIC_SCRATCH_BYTES (1 << 20)
+
+/* zero_shard_step for callers that cannot allocate device memory.  This entry
+ * point has no counterpart on the ZeRO pages; it exists for code that runs
+ * where a cudaMalloc is not available or not allowed -- inside a framework
+ * whose caching allocator owns the whole device and forbids raw allocations
+ * beside it, in plug-in or embedded runtimes that are handed buffers but no
+ * allocator, or in step loops where an allocation (which may synchronise the
+ * device) is not acceptable.
+ *
+ * Behaviour, arguments and errors are those of zero_shard_step, except that
+ * args->workspace and args->workspace_bytes are ignored: the scratch (the
+ * per-step header and the fp64 norm partials) lives in one static device
+ * array of ZERO_STATIC_SCRATCH_BYTES inside the library.  No call allocates
+ * or frees device memory.
+ *   - Limit: SPECULATIVE calls need 256 bytes; TWO_PASS and STASH calls need
+ *     256 bytes plus 8 per statistics block (at most 2048 blocks per
+ *     bucket), i.e. up to 63 full-size buckets.  A call needing more returns
+ *     ZERO_ERR_WORKSPACE before anything is launched (zero_workspace_bytes
+ *     tells the size in advance).
+ *   - The first call on a device resolves the array's device address with
+ *     that device current and caches it; make that first call before any
+ *     stream capture begins.
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents.  Each call rewrites the header and every partial it
+ *     reads before reading it, so nothing has to start at zero.  Calls whose
+ *     GPU work overlaps (unordered streams, or host threads racing on one
+ *     device) race on the array and corrupt each other's overflow flag and
+ *     norm: order them, e.g. on one stream. */
+ZERO_API zero_status zero_shard_step_static_scratch(const zero_plan_t* plan, const zero_hparams* hp,
+                                                    const zero_step_args* args, void* stream);
+
 /* Gather-assembly (the stage-3 all-gather seen by one rank): for every owner
  * r whose shard_ptrs[r] (host array of nd device pointers) is not NULL,
  * copies its fp16 shard [0, real_len_r) into params_full[r * L ...].

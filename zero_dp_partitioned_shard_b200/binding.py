@@ -33,6 +33,8 @@ ZERO_MODE_STASH = 2
 ZERO_GRADS_FULL = 0
 ZERO_GRADS_PER_OWNER = 1
 
+ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
+
 OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (40 bytes used)
 RESULT_BYTES = 64      # device allocation for zero_step_result (32 bytes used)
 
@@ -114,6 +116,7 @@ SIGNATURES = {
     "zero_opt_state_init": (_S, [_P, _P]),
     "zero_workspace_bytes": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), C.POINTER(C.c_size_t)]),
     "zero_shard_step": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
+    "zero_shard_step_static_scratch": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, _P]),
     "zero_abi_version": (C.c_int32, []),
@@ -216,6 +219,12 @@ def zero_workspace_bytes(plan: int, hp: HParams, args: StepArgs) -> int:
 
 def zero_shard_step(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
     _check(lib().zero_shard_step(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step")
+
+
+def zero_shard_step_static_scratch(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
+    """zero_shard_step with the library's static device scratch (args.workspace ignored)."""
+    _check(lib().zero_shard_step_static_scratch(plan, C.byref(hp), C.byref(args), stream),
+           "zero_shard_step_static_scratch")
 
 
 def zero_gather_params(plan: int, shard_ptrs, params_full: int, stream: int = 0) -> None:
