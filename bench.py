@@ -74,6 +74,31 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     return alg, moved
 
 
+def profiled_traffic(nd: int, mode: int, owned: int):
+    """DRAM bytes (read + write) of one update-kernel launch, from a committed
+    ncu summary under profiles/ that was captured on the current kernel source
+    with the same Nd and mode, scaled to this launch by its parameters.  None
+    when no such summary exists (for instance after the kernel changed)."""
+    import glob
+    import hashlib
+    src = os.path.join(ROOT, "zero_dp_partitioned_shard_b200", "csrc", "kernels.cu")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None, None
+    mode_name = {0: "speculative", 1: "two_pass", 2: "stash"}[mode]
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        kv = {}
+        for line in open(path):
+            if ":" in line and not line.startswith(("|", " ", "#")):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if (kv.get("kernels_cu_sha256_prefix") == sha and kv.get("traffic_nd") == str(nd)
+                and kv.get("traffic_mode") == mode_name and "traffic_bytes_per_param" in kv):
+            return float(kv["traffic_bytes_per_param"]) * owned, os.path.relpath(path, ROOT)
+    return None, None
+
+
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -229,14 +254,22 @@ def _dist():
     return world, rank, local
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank scalar over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(owned: int, steps: int, ms_local: float, world: int, device: str = "cuda"):
+    """Whole-job throughput: parameters updated by all ranks over the slowest
+    rank's device time.  Returns (ms_max, params_per_second)."""
+    ms_max = max_over_ranks(ms_local, world, device)
+    return ms_max, world * owned * steps / (ms_max / 1e3)
 
 
 def _barrier(world: int):
@@ -372,10 +405,9 @@ def main():
     clk = clocks.stop()
     _barrier(world)
     ms = t_start.elapsed_time(t_end)
-    ms_max = _max_over_ranks(ms, world)
+    ms_max, value = aggregate(bench.owned, args.steps, ms, world)
     k_ms = statistics.mean(a.elapsed_time(b) for a, b in k_events)
-    k_ms_max = _max_over_ranks(k_ms, world)
-    value = world * bench.owned * args.steps / (ms_max / 1e3)
+    k_ms_max = max_over_ranks(k_ms, world)
     res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
 
     # --- end to end through the C ABI, host buffers ---
@@ -401,8 +433,8 @@ def main():
                 B.step_result_from_bytes(r_host.numpy().tobytes())  # the caller reads the result
             e1.record()
             torch.cuda.synchronize()
-            e_ms = _max_over_ranks(e0.elapsed_time(e1), world)
-            e2e = {"value": world * bench.owned * args.e2e_steps / (e_ms / 1e3), "unit": UNIT,
+            e_ms, e_value = aggregate(bench.owned, args.e2e_steps, e0.elapsed_time(e1), world)
+            e2e = {"value": e_value, "unit": UNIT,
                    "h2d_bytes_per_step": bench.grad_bytes, "d2h_bytes_per_step": B.RESULT_BYTES,
                    "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps}
             del g_host
@@ -411,6 +443,7 @@ def main():
 
     peak, peak_kind = measured_hbm_peak()
     achieved = bench.owned * alg / (k_ms_max / 1e3) / 1e9
+    traffic, traffic_src = profiled_traffic(wl["nd"], wl["mode"], bench.owned)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -424,7 +457,7 @@ def main():
                          f"{bench.owned * moved / 1e9:.1f} GB moved per step",
                    "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                      "kernel": "zs_update_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
                      "alg_bytes_per_launch": bench.owned * alg},
