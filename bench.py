@@ -63,7 +63,7 @@ def _workloads():
                  "(L=117,187,584) with 64 fp16 contributions, speculative mode",
             sizes=None, psi=7_500_000_000, nd=64, stage=3, align=256, bucket=0, S=1.0, wd=0.0,
             clip=0.0, mode=B.ZERO_MODE_SPECULATIVE, layout=B.ZERO_GRADS_PER_OWNER,
-            owner_first=0, owner_count=1),
+            owner_first=0, owner_count=1, assemble=True),
     }
 
 
@@ -72,6 +72,13 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     alg = 2 * nd + 26  # Nd fp16 reads, master/m/v read+write (24), fp16 write (2)
     moved = {0: alg, 1: 4 * nd + 26, 2: 2 * nd + 34}[mode]
     return alg, moved
+
+
+def update_launch_bytes(nd: int, mode: int) -> int:
+    """Algorithmic bytes per parameter of the update kernel's own launch: the
+    fused kernel reads the Nd contributions (speculative, two-pass) or the
+    4-byte stash (stash), plus master/m/v read and write and the fp16 write."""
+    return (4 if mode == 2 else 2 * nd) + 26
 
 
 def profiled_traffic(nd: int, mode: int, owned: int):
@@ -218,6 +225,18 @@ class Bench:
             exp_avg_sq=tuple(ptr(t) for t in self.exp_avg_sq), params=self.params.data_ptr(),
             grad_stash=ptr(self.stash), opt_state=self.opt_state.data_ptr(),
             result=self.result.data_ptr())
+        # stage-3 view: after its own update the rank assembles the full fp16
+        # buffer from the other owners' (seeded) parameter shards
+        self.shards, self.shard_ptrs, self.assembled = None, None, 0
+        if wl.get("assemble"):
+            others = [r for r in range(self.nd) if not (o0 <= r < o0 + oc)]
+            self.shards = torch.empty(len(others), L, dtype=torch.float16, device=dev)
+            for k, r in enumerate(others):
+                synth.fill_normal_(self.shards[k], seed=seed * 1000 + 500 + r, std=0.02)
+            self.shard_ptrs = [0] * self.nd
+            for k, r in enumerate(others):
+                self.shard_ptrs[r] = self.shards[k].data_ptr()
+            self.assembled = sum(max(0, min(L, psi - r * L)) for r in others)
         ws_bytes = B.zero_workspace_bytes(self.plan, self.hp, self.args)
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.args.workspace = self.workspace.data_ptr()
@@ -233,6 +252,8 @@ class Bench:
             self.args.timing_events[0] = None
             self.args.timing_events[1] = None
         self.B.zero_shard_step(self.plan, self.hp, self.args, self.stream)
+        if self.shard_ptrs is not None:
+            self.B.zero_gather_params(self.plan, self.shard_ptrs, self.params.data_ptr(), self.stream)
 
     def close(self):
         self.B.zero_plan_destroy(self.plan)
@@ -346,6 +367,72 @@ def run_reference(args, wl_name: str, wl: dict):
     return 0
 
 
+SWEEP_PSI = [1 << 20, 16 << 20, 256 << 20, 1 << 30, 2 << 30]
+SWEEP_ND = [1, 2, 8, 64]
+
+
+def sweep_workload(psi: int, nd: int, stage: int, free_bytes: int) -> dict:
+    """One sweep point: speculative, no clipping; stage 1 = full gradients in one
+    pass, stage 2 = the same in 8 buckets, stage 3 = per-owner contributions.
+    All Nd owners are simulated when Psi*(2*Nd + 26) bytes fit in 80 % of free
+    HBM; otherwise owner 0's view (the same bytes per parameter)."""
+    from zero_dp_partitioned_shard_b200 import binding as B
+    full_bytes = psi * (2 * nd + 26) + (1 << 28)
+    one_owner = full_bytes > 0.8 * free_bytes
+    bucket = 0
+    if stage == 2:
+        bucket = -(-psi // (8 * 256)) * 256
+    return dict(desc=f"sweep psi={psi} nd={nd} stage={stage}" + (" owner-0 view" if one_owner else ""),
+                sizes=None, psi=psi, nd=nd, stage=stage, align=256, bucket=bucket, S=1.0, wd=0.0,
+                clip=0.0, mode=B.ZERO_MODE_SPECULATIVE,
+                # a one-owner view holds only its own slice of each rank's gradient
+                layout=B.ZERO_GRADS_PER_OWNER if (stage == 3 or one_owner) else B.ZERO_GRADS_FULL,
+                owner_first=0, owner_count=1 if one_owner else None)
+
+
+def run_sweep(args) -> int:
+    """Update-kernel GB/s against bytes per parameter over the sweep grid; one
+    JSON line per point (measurement mode, not the benchmark line)."""
+    import torch
+    world, rank, local = _dist()
+    peak, peak_kind = measured_hbm_peak()
+    for psi in SWEEP_PSI:
+        for nd in SWEEP_ND:
+            for stage in (1, 2, 3):
+                torch.cuda.empty_cache()
+                free, _ = torch.cuda.mem_get_info()
+                wl = sweep_workload(psi, nd, stage, free)
+                bn = Bench(wl, None, seed=7)
+                for _ in range(args.warmup):
+                    bn.step()
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(args.steps)]
+                for a, b in ev:
+                    a.record()
+                    b.record()
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                t0.record()
+                for k in range(args.steps):
+                    bn.step(ev[k])
+                t1.record()
+                torch.cuda.synchronize()
+                k_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+                step_ms = t0.elapsed_time(t1) / args.steps
+                alg = update_launch_bytes(nd, wl["mode"])
+                gbs = bn.owned * alg / (k_ms / 1e3) / 1e9
+                if rank == 0:
+                    print(json.dumps({"sweep": True, "psi": psi, "nd": nd, "stage": stage,
+                                      "view": "owner0" if wl["owner_count"] == 1 else "all owners",
+                                      "owned": bn.owned, "bytes_per_param": alg,
+                                      "kernel_ms": k_ms, "step_ms": step_ms, "gbs": gbs,
+                                      "frac": gbs / peak, "peak": peak, "peak_kind": peak_kind,
+                                      "params_per_s": bn.owned / (step_ms / 1e3)}), flush=True)
+                bn.close()
+                del bn
+    return 0
+
+
 def _psi_of(wl):
     return sum(wl["sizes"]()) if wl.get("sizes") else wl["psi"]
 
@@ -364,9 +451,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-sample", type=int, default=1 << 22)
     ap.add_argument("--ref-sample", type=int, default=1 << 21)
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure the Psi x Nd x stage grid (one JSON line per point)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        return run_sweep(args)
     wls = _workloads()
     if args.workload not in wls:
         ap.error(f"unknown workload {args.workload}; choose from {sorted(wls)}")
@@ -442,7 +533,8 @@ def main():
             e2e = {"value": None, "unit": UNIT, "skipped": "host memory below 2.5x the gradient bytes"}
 
     peak, peak_kind = measured_hbm_peak()
-    achieved = bench.owned * alg / (k_ms_max / 1e3) / 1e9
+    k_bytes = bench.owned * update_launch_bytes(wl["nd"], wl["mode"])
+    achieved = k_bytes / (k_ms_max / 1e3) / 1e9
     traffic, traffic_src = profiled_traffic(wl["nd"], wl["mode"], bench.owned)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -452,7 +544,9 @@ def main():
                    "nd": wl["nd"], "stage": wl["stage"], "owned_params_per_gpu": bench.owned,
                    "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
                    "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
-                   "step_gbs_alg": bench.owned * alg / (ms_max / args.steps / 1e3) / 1e9,
+                   "assembled_params": bench.assembled,
+                   "step_gbs_alg": (bench.owned * alg + 4 * bench.assembled)
+                                   / (ms_max / args.steps / 1e3) / 1e9,
                    "l2": "inputs larger than L2 (no flush): "
                          f"{bench.owned * moved / 1e9:.1f} GB moved per step",
                    "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
@@ -460,7 +554,7 @@ def main():
                      "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
                      "kernel": "zs_update_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
-                     "alg_bytes_per_launch": bench.owned * alg},
+                     "alg_bytes_per_launch": k_bytes},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
