@@ -371,20 +371,20 @@ SWEEP_PSI = [1 << 20, 16 << 20, 256 << 20, 1 << 30, 2 << 30]
 SWEEP_ND = [1, 2, 8, 64]
 
 
-def sweep_workload(psi: int, nd: int, stage: int, free_bytes: int) -> dict:
+def sweep_workload(psi: int, nd: int, stage: int, free_bytes: int, mode: int = 0) -> dict:
     """One sweep point: speculative, no clipping; stage 1 = full gradients in one
     pass, stage 2 = the same in 8 buckets, stage 3 = per-owner contributions.
     All Nd owners are simulated when Psi*(2*Nd + 26) bytes fit in 80 % of free
     HBM; otherwise owner 0's view (the same bytes per parameter)."""
     from zero_dp_partitioned_shard_b200 import binding as B
-    full_bytes = psi * (2 * nd + 26) + (1 << 28)
+    full_bytes = psi * (2 * nd + 26 + (4 if mode == B.ZERO_MODE_STASH else 0)) + (1 << 28)
     one_owner = full_bytes > 0.8 * free_bytes
     bucket = 0
     if stage == 2:
         bucket = -(-psi // (8 * 256)) * 256
     return dict(desc=f"sweep psi={psi} nd={nd} stage={stage}" + (" owner-0 view" if one_owner else ""),
                 sizes=None, psi=psi, nd=nd, stage=stage, align=256, bucket=bucket, S=1.0, wd=0.0,
-                clip=0.0, mode=B.ZERO_MODE_SPECULATIVE,
+                clip=1.0 if mode != B.ZERO_MODE_SPECULATIVE else 0.0, mode=mode,
                 # a one-owner view holds only its own slice of each rank's gradient
                 layout=B.ZERO_GRADS_PER_OWNER if (stage == 3 or one_owner) else B.ZERO_GRADS_FULL,
                 owner_first=0, owner_count=1 if one_owner else None)
@@ -396,12 +396,15 @@ def run_sweep(args) -> int:
     import torch
     world, rank, local = _dist()
     peak, peak_kind = measured_hbm_peak()
-    for psi in SWEEP_PSI:
-        for nd in SWEEP_ND:
-            for stage in (1, 2, 3):
+    ints = lambda text, default: [int(x) for x in text.split(",")] if text else default
+    modes = {"speculative": 0, "two_pass": 1, "stash": 2}
+    for psi in ints(args.sweep_psi, SWEEP_PSI):
+        for nd in ints(args.sweep_nd, SWEEP_ND):
+          for mode_name in (args.sweep_mode or "speculative").split(","):
+            for stage in ints(args.sweep_stage, [1, 2, 3]):
                 torch.cuda.empty_cache()
                 free, _ = torch.cuda.mem_get_info()
-                wl = sweep_workload(psi, nd, stage, free)
+                wl = sweep_workload(psi, nd, stage, free, modes[mode_name])
                 bn = Bench(wl, None, seed=7)
                 for _ in range(args.warmup):
                     bn.step()
@@ -423,6 +426,7 @@ def run_sweep(args) -> int:
                 gbs = bn.owned * alg / (k_ms / 1e3) / 1e9
                 if rank == 0:
                     print(json.dumps({"sweep": True, "psi": psi, "nd": nd, "stage": stage,
+                                      "mode": mode_name,
                                       "view": "owner0" if wl["owner_count"] == 1 else "all owners",
                                       "owned": bn.owned, "bytes_per_param": alg,
                                       "kernel_ms": k_ms, "step_ms": step_ms, "gbs": gbs,
@@ -453,6 +457,10 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=1 << 21)
     ap.add_argument("--sweep", action="store_true",
                     help="measure the Psi x Nd x stage grid (one JSON line per point)")
+    ap.add_argument("--sweep-psi", default="", help="comma-separated Psi values (default: the grid)")
+    ap.add_argument("--sweep-nd", default="", help="comma-separated Nd values")
+    ap.add_argument("--sweep-stage", default="", help="comma-separated stages")
+    ap.add_argument("--sweep-mode", default="", help="speculative,two_pass,stash (default speculative)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 1
+#define ZERO_SHARD_ABI_VERSION 2
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -78,7 +78,7 @@ typedef int32_t zero_status;
 #define ZERO_ERR_ALIGNMENT 2   /* a pointer is not aligned to its element size  */
 #define ZERO_ERR_CUDA 3        /* a CUDA runtime call or launch failed          */
 #define ZERO_ERR_WORKSPACE 4   /* workspace missing or smaller than required    */
-#define ZERO_ERR_TIMEOUT 5     /* reserved: no kernel of this library waits     */
+#define ZERO_ERR_TIMEOUT 5     /* a bounded device-side wait expired (reported in zero_step_result.status) */
 #define ZERO_ERR_UNSUPPORTED 6 /* combination not available (e.g. clip + speculative) */
 
 /* ---- enumerations --------------------------------------------------------- */
@@ -201,6 +201,11 @@ typedef struct zero_step_result {
     int64_t skipped;   /* zero_opt_state.skipped after the call */
     float clip_coef;   /* coefficient applied (1 when not clipping) */
     int32_t overflow;  /* 1: a non-finite gradient was seen, nothing was updated */
+    int32_t status;    /* ZERO_OK, or ZERO_ERR_TIMEOUT if a pipeline wait inside a
+                          kernel gave up (a fault, never expected): SPECULATIVE
+                          then keeps the previous state as on overflow; in
+                          TWO_PASS / STASH the update is incomplete */
+    int32_t reserved;
 } zero_step_result;
 
 /* ---- the step ---------------------------------------------------------------------- */

@@ -36,7 +36,7 @@ ZERO_GRADS_PER_OWNER = 1
 ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
 
 OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (40 bytes used)
-RESULT_BYTES = 64      # device allocation for zero_step_result (32 bytes used)
+RESULT_BYTES = 64      # device allocation for zero_step_result (40 bytes used)
 
 
 class ZeroError(RuntimeError):
@@ -79,7 +79,8 @@ class OptState(C.Structure):
 
 class StepResult(C.Structure):
     _fields_ = [("grad_norm", C.c_double), ("t", C.c_int64), ("skipped", C.c_int64),
-                ("clip_coef", C.c_float), ("overflow", C.c_int32)]
+                ("clip_coef", C.c_float), ("overflow", C.c_int32), ("status", C.c_int32),
+                ("reserved", C.c_int32)]
 
 
 class HParams(C.Structure):
@@ -139,7 +140,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 1:
+        if L.zero_abi_version() != 2:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib

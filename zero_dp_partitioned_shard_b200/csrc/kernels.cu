@@ -198,6 +198,7 @@ __global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float bet
     const double b1 = __dmul_rn(st->beta1_pow, (double)beta1);
     const double b2 = __dmul_rn(st->beta2_pow, (double)beta2);
     ws->overflow = 0u;
+    ws->error = 0u;
     ws->skip = 0;
     ws->cur = st->cur & 1;
     ws->bc1 = __double2float_rn(__dsub_rn(1.0, b1));
@@ -213,6 +214,28 @@ __global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float bet
 // ---------------------------------------------------------------------------
 // K1: fused reduce + unscale (+ overflow) + clip + Adam + fp16 cast
 // ---------------------------------------------------------------------------
+
+// One element, scalar loads and stores; returns true if its gradient is not
+// finite (only meaningful when the reduced gradient is computed here).
+template <int SRC>
+__device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg, int64_t e, const AdamK& k,
+                                              const float* p_in, const float* m_in, const float* v_in,
+                                              float* p_out, float* m_out, float* v_out)
+{
+    const int64_t so = sg.s_off + e;
+    float g;
+    if (SRC == kSrcStash)
+        g = a.stash[so];
+    else
+        g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
+    float p = p_in[so], m = m_in[so], v = v_in[so];
+    adam_update(__fmul_rn(g, k.clip), p, m, v, k);
+    p_out[so] = p;
+    m_out[so] = m;
+    v_out[so] = v;
+    a.params[sg.p_off + e] = f2h(p);
+    return !isfinite(g);
+}
 
 template <int SRC, bool VEC>
 __global__ void __launch_bounds__(kThreads)
@@ -270,25 +293,333 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8(p));
         }
         // scalar elements: everything (VEC = false) or the < 8 tail
-        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr) {
-            const int64_t so = sg.s_off + e;
-            float g;
-            if (SRC == kSrcStash)
-                g = a.stash[so];
-            else
-                g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
-            if (kSpec)
-                bad |= !isfinite(g);
-            float p = p_in[so], m = m_in[so], v = v_in[so];
-            adam_update(__fmul_rn(g, k.clip), p, m, v, k);
-            p_out[so] = p;
-            m_out[so] = m;
-            v_out[so] = v;
-            a.params[sg.p_off + e] = f2h(p);
-        }
+        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr)
+            bad |= update_scalar<SRC>(a, sg, e, k, p_in, m_in, v_in, p_out, m_out, v_out);
     }
     if (kSpec)
         flag_nonfinite(bad, &a.ws->overflow);
+}
+
+// ---------------------------------------------------------------------------
+// K1, bulk-copy pipeline: the same per-element arithmetic, with the operands
+// staged through shared memory.  One producer thread streams each tile of
+// master/m/v and of the Nd rank contributions (or the stash) into a ring of
+// shared-memory stages with 1-D cp.async.bulk copies that complete on an
+// mbarrier; eight consumer warps wait for a stage, compute from shared memory,
+// store straight to global memory and release the stage.  Loads in flight no
+// longer depend on registers or occupancy: (stages - 1) tiles per CTA are
+// always on their way.  Every wait is bounded; a wait that expires sets the
+// workspace error word and the result's status, and the kernel exits after
+// waiting (bounded) for its own copies.
+// ---------------------------------------------------------------------------
+
+constexpr int kPipeConsumerWarps = 8;
+constexpr int kPipeConsumers = kPipeConsumerWarps * 32;
+constexpr int kPipeThreads = kPipeConsumers + 32; // + the producer warp
+constexpr long long kWaitBudgetCycles = 1ll << 31; // ~1 s: far beyond any memory latency
+constexpr int kPipeHeaderBytes = 1024;           // mbarriers + tile table, before the ring
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_addr(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of the given parity; false if the budget ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_test(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity))
+        if (clock64() - t0 > kWaitBudgetCycles)
+            return false;
+    return true;
+}
+
+// global -> shared bulk copy of `bytes` (multiple of 16, both ends 16-byte
+// aligned) completing as transaction bytes on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void lds_f(const float* p, float f[N])
+{
+    if (N == 8) {
+        const float4 x = reinterpret_cast<const float4*>(p)[0];
+        const float4 y = reinterpret_cast<const float4*>(p)[1];
+        f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+        f[4] = y.x; f[5] = y.y; f[6] = y.z; f[7] = y.w;
+    } else if (N == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(p);
+        f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    } else if (N == 2) {
+        const float2 x = *reinterpret_cast<const float2*>(p);
+        f[0] = x.x; f[1] = x.y;
+    } else {
+        f[0] = p[0];
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void lds_h(const uint16_t* p, float f[N])
+{
+    if (N == 8) {
+        unpack_h8(*reinterpret_cast<const uint4*>(p), f);
+    } else if (N == 4) {
+        const uint2 x = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
+        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    } else if (N == 2) {
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(p));
+        f[0] = a.x; f[1] = a.y;
+    } else {
+        f[0] = h2f(p[0]);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void stg_f(float* p, const float f[N])
+{
+    if (N == 8)
+        st_f8(p, f);
+    else if (N == 4)
+        __stcs(reinterpret_cast<float4*>(p), make_float4(f[0], f[1], f[2], f[3]));
+    else if (N == 2)
+        __stcs(reinterpret_cast<float2*>(p), make_float2(f[0], f[1]));
+    else
+        __stcs(p, f[0]);
+}
+
+template <int N>
+__device__ __forceinline__ void stg_h(uint16_t* p, const float f[N])
+{
+    if (N == 8) {
+        __stcs(reinterpret_cast<uint4*>(p), pack_h8(f));
+    } else if (N == 4) {
+        __half2 h0 = __floats2half2_rn(f[0], f[1]), h1 = __floats2half2_rn(f[2], f[3]);
+        uint2 x;
+        x.x = *reinterpret_cast<uint32_t*>(&h0);
+        x.y = *reinterpret_cast<uint32_t*>(&h1);
+        __stcs(reinterpret_cast<uint2*>(p), x);
+    } else if (N == 2) {
+        __half2 h0 = __floats2half2_rn(f[0], f[1]);
+        __stcs(reinterpret_cast<unsigned int*>(p), *reinterpret_cast<unsigned int*>(&h0));
+    } else {
+        p[0] = f2h(f[0]);
+    }
+}
+
+// tile g of the launch -> segment and offset, through the per-CTA tile table
+__device__ __forceinline__ int tile_segment(const int64_t* first_tile, int count, int64_t g)
+{
+    int s = 0;
+    while (s + 1 < count && g >= first_tile[s + 1])
+        ++s;
+    return s;
+}
+
+template <int SRC, int EPT>
+__global__ void __launch_bounds__(kPipeThreads, 2)
+zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages)
+{
+    constexpr bool kSpec = SRC == kSrcGradsSpeculative;
+    constexpr int T = kPipeConsumers * EPT; // elements per tile
+    WsHeader* ws = a.ws;
+    if (!kSpec && ws->skip)
+        return; // uniform: the whole step is skipped
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + stages;
+    int64_t* first_tile = reinterpret_cast<int64_t*>(smem + 256); // [count + 1]
+    unsigned char* ring = smem + kPipeHeaderBytes;
+    const int src_bytes = SRC == kSrcStash ? 4 : 2 * a.nd;        // per element
+    const int stage_bytes = T * (12 + src_bytes);
+
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        for (int s = 0; s < segs.count; ++s) {
+            first_tile[s] = acc;
+            acc += ((segs.seg[s].n >> 3) * 8 + T - 1) / T;
+        }
+        first_tile[segs.count] = acc;
+        for (int i = 0; i < stages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kPipeConsumerWarps);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    const int64_t n_tiles = first_tile[segs.count];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cur = kSpec ? ws->cur : 0;
+    const int nxt = kSpec ? cur ^ 1 : 0;
+    const float* p_in = cur ? a.master[1] : a.master[0];
+    const float* m_in = cur ? a.exp_avg[1] : a.exp_avg[0];
+    const float* v_in = cur ? a.exp_avg_sq[1] : a.exp_avg_sq[0];
+    float* p_out = nxt ? a.master[1] : a.master[0];
+    float* m_out = nxt ? a.exp_avg[1] : a.exp_avg[0];
+    float* v_out = nxt ? a.exp_avg_sq[1] : a.exp_avg_sq[0];
+    bool failed = false;
+
+    if (warp == kPipeConsumerWarps) {
+        // ---- producer warp: lane 0 claims a free stage and announces its
+        // bytes; the tile's copies (3 state arrays + the source rows) are then
+        // issued by all 32 lanes at once ----
+        const int n_copies = 3 + (SRC == kSrcStash ? 1 : a.nd);
+        int it = 0;
+        for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
+            const int st = it % stages;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(&empty[st], ((it / stages) & 1) ^ 1);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                failed = true;
+                break;
+            }
+            const int si = tile_segment(first_tile, segs.count, g);
+            const Seg& sg = segs.seg[si];
+            const int64_t e0 = (g - first_tile[si]) * T;
+            const int64_t nv = (sg.n >> 3) * 8;
+            const uint32_t n = (uint32_t)(nv - e0 < T ? nv - e0 : T);
+            unsigned char* buf = ring + (size_t)st * stage_bytes;
+            if (lane == 0)
+                mbar_arrive_expect_tx(&full[st], n * (12u + (uint32_t)src_bytes));
+            __syncwarp();
+            const int64_t so = sg.s_off + e0;
+            for (int j = lane; j < n_copies; j += 32) {
+                if (j < 3) {
+                    const float* src = j == 0 ? p_in : (j == 1 ? m_in : v_in);
+                    bulk_load(buf + j * (T * 4), src + so, n * 4, &full[st]);
+                } else if (SRC == kSrcStash) {
+                    bulk_load(buf + T * 12, a.stash + so, n * 4, &full[st]);
+                } else {
+                    const int r = j - 3;
+                    bulk_load(buf + T * 12 + r * (T * 2), a.grads + sg.g_off + e0 + (int64_t)r * sg.g_rstride,
+                              n * 2, &full[st]);
+                }
+            }
+        }
+        // every copy issued lands before the producer may leave the CTA
+        if (lane == 0) {
+            const int issued = it;
+            for (int st = 0; st < stages && st < issued; ++st) {
+                const int last = issued - 1 - ((issued - 1 - st) % stages); // last use of stage st
+                if (!mbar_wait(&full[st], (last / stages) & 1))
+                    failed = true;
+            }
+        }
+    } else {
+        // ---- consumers ----
+        const AdamK k = load_consts(a, ws, !kSpec);
+        const int c = threadIdx.x; // 0 .. kPipeConsumers-1
+        bool bad = false;
+        int it = 0;
+        for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
+            const int st = it % stages;
+            const bool ok = mbar_wait(&full[st], (it / stages) & 1);
+            if (!__all_sync(0xffffffffu, ok)) {
+                failed = true;
+                break;
+            }
+            const int si = tile_segment(first_tile, segs.count, g);
+            const Seg& sg = segs.seg[si];
+            const int64_t e0 = (g - first_tile[si]) * T;
+            const int64_t nv = (sg.n >> 3) * 8;
+            const int n = (int)(nv - e0 < T ? nv - e0 : T);
+            const int i0 = c * EPT; // this thread's first element in the tile
+            if (i0 < n) {
+                const unsigned char* buf = ring + (size_t)st * stage_bytes;
+                float p[EPT], m[EPT], v[EPT], gr[EPT];
+                lds_f<EPT>(reinterpret_cast<const float*>(buf) + i0, p);
+                lds_f<EPT>(reinterpret_cast<const float*>(buf + T * 4) + i0, m);
+                lds_f<EPT>(reinterpret_cast<const float*>(buf + T * 8) + i0, v);
+                if (SRC == kSrcStash) {
+                    lds_f<EPT>(reinterpret_cast<const float*>(buf + T * 12) + i0, gr);
+                } else {
+                    const uint16_t* gs = reinterpret_cast<const uint16_t*>(buf + T * 12) + i0;
+                    lds_h<EPT>(gs, gr);
+                    for (int r = 1; r < a.nd; ++r) {
+                        float f[EPT];
+                        lds_h<EPT>(gs + r * T, f);
+#pragma unroll
+                        for (int q = 0; q < EPT; ++q)
+                            gr[q] = __fadd_rn(gr[q], f[q]);
+                    }
+#pragma unroll
+                    for (int q = 0; q < EPT; ++q)
+                        gr[q] = __fmul_rn(gr[q], a.inv);
+                }
+                if (kSpec) {
+#pragma unroll
+                    for (int q = 0; q < EPT; ++q)
+                        bad |= !isfinite(gr[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < EPT; ++q)
+                    adam_update(__fmul_rn(gr[q], k.clip), p[q], m[q], v[q], k);
+                const int64_t so = sg.s_off + e0 + i0;
+                stg_f<EPT>(p_out + so, p);
+                stg_f<EPT>(m_out + so, m);
+                stg_f<EPT>(v_out + so, v);
+                stg_h<EPT>(a.params + sg.p_off + e0 + i0, p);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
+        }
+        // the < 8-element tail of each segment, scalar
+        const int64_t gtid = (int64_t)blockIdx.x * kPipeConsumers + c;
+        if (!failed) {
+            for (int si = 0; si < segs.count; ++si) {
+                const Seg& sg = segs.seg[si];
+                const int64_t e = (sg.n >> 3) * 8 + gtid;
+                if (e < sg.n)
+                    bad |= update_scalar<SRC>(a, sg, e, k, p_in, m_in, v_in, p_out, m_out, v_out);
+            }
+        }
+        if (kSpec)
+            flag_nonfinite(bad, &ws->overflow);
+    }
+    if (failed) {
+        atomicOr(&ws->error, 1u);
+        if (a.result)
+            a.result->status = ZERO_ERR_TIMEOUT;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -400,6 +731,8 @@ zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_no
         res->skipped = st->skipped;
         res->clip_coef = clip;
         res->overflow = skip ? 1 : 0;
+        res->status = ZERO_OK;
+        res->reserved = 0;
     }
 }
 
@@ -433,7 +766,8 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
                  zero_opt_state* st, zero_step_result* res)
 {
     const WsHeader* ws = a.ws;
-    const bool over = ws->overflow != 0u;
+    const bool fault = ws->error != 0u;
+    const bool over = ws->overflow != 0u || fault;
     const int cur = ws->cur;
     if (bookkeeping && blockIdx.x == 0 && threadIdx.x == 0) {
         if (!over) {
@@ -449,7 +783,9 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
             res->t = st->t;
             res->skipped = st->skipped;
             res->clip_coef = 1.0f;
-            res->overflow = over ? 1 : 0;
+            res->overflow = ws->overflow != 0u ? 1 : 0;
+            res->status = fault ? ZERO_ERR_TIMEOUT : ZERO_OK;
+            res->reserved = 0;
         }
     }
     if (!over)
@@ -593,8 +929,99 @@ static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, cud
     return cudaGetLastError();
 }
 
+// Shape of the pipelined update for a given source: elements per consumer
+// thread (tile = 256 x EPT), ring stages and CTAs per SM.  A stage holds one
+// tile of master/m/v plus the tile's source bytes; it is kept <= 48 KB for
+// EPT > 1, and two CTAs share an SM when three or more stages fit in half of
+// its shared memory.
+struct PipeShape {
+    int ept = 0, stages = 0, ctas_per_sm = 0, smem = 0;
+};
+
+static bool pipe_shape(int src, int nd, PipeShape* ps)
+{
+    const int e = 12 + (src == kSrcStash ? 4 : 2 * nd);
+    const int ept = 2048 * e <= 32 * 1024 ? 8
+                  : (1024 * e <= 48 * 1024 ? 4 : (512 * e <= 48 * 1024 ? 2 : (256 * e <= 72 * 1024 ? 1 : 0)));
+    if (!ept)
+        return false;
+    const int stage = kPipeConsumers * ept * e;
+    int ctas = 2, stages = (110 * 1024 - kPipeHeaderBytes) / stage;
+    if (stages < 3) {
+        ctas = 1;
+        stages = (220 * 1024 - kPipeHeaderBytes) / stage;
+    }
+    stages = stages > 8 ? 8 : stages;
+    if (stages < 2)
+        return false;
+    ps->ept = ept;
+    ps->stages = stages;
+    ps->ctas_per_sm = ctas;
+    ps->smem = kPipeHeaderBytes + stages * stage;
+    return true;
+}
+
+static std::map<std::pair<const void*, int>, int> g_smem_set; // (kernel, device) -> bytes allowed
+
+template <int SRC, int EPT>
+static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+{
+    auto kernel = zs_update_pipe_kernel<SRC, EPT>;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || (e = device_sms(&sms)) != cudaSuccess)
+        return e;
+    const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_smem_set.find(key);
+        if (it == g_smem_set.end() || it->second < ps.smem) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024 + kPipeHeaderBytes);
+            if (e != cudaSuccess)
+                return e;
+            g_smem_set[key] = 220 * 1024 + kPipeHeaderBytes;
+        }
+    }
+    int64_t tiles = 0;
+    const int T = kPipeConsumers * EPT;
+    for (int i = 0; i < segs.count; ++i)
+        tiles += ((segs.seg[i].n >> 3) * 8 + T - 1) / T;
+    int64_t grid = (int64_t)sms * ps.ctas_per_sm;
+    grid = tiles < grid ? tiles : grid;
+    grid = grid < 1 ? 1 : grid;
+    kernel<<<(unsigned)grid, kPipeThreads, ps.smem, s>>>(a, segs, ps.stages);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <int SRC>
+static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+{
+    switch (ps.ept) {
+    case 8: return launch_pipe_t<SRC, 8>(a, segs, ps, s);
+    case 4: return launch_pipe_t<SRC, 4>(a, segs, ps, s);
+    case 2: return launch_pipe_t<SRC, 2>(a, segs, ps, s);
+    default: return launch_pipe_t<SRC, 1>(a, segs, ps, s);
+    }
+}
+
+// The bulk-copy pipeline pays off where a parameter carries few bytes (the
+// stash source, Nd <= 2: measured 0.87-0.88 of the copy bandwidth against
+// 0.85-0.86 for the register path); from Nd = 4 up the register path, whose
+// groups of 8 rank loads keep more bytes in flight per thread, is faster
+// (0.95-1.02 against 0.64-0.95).
+static bool use_pipeline(int src, int nd) { return src == kSrcStash || nd <= 2; }
+
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, cudaStream_t s)
 {
+    PipeShape ps;
+    if (vec && use_pipeline(src, a.nd) && pipe_shape(src, a.nd, &ps)) {
+        switch (src) {
+        case kSrcGradsSpeculative: return launch_pipe<kSrcGradsSpeculative>(a, segs, ps, s);
+        case kSrcGradsInPlace: return launch_pipe<kSrcGradsInPlace>(a, segs, ps, s);
+        default: return launch_pipe<kSrcStash>(a, segs, ps, s);
+        }
+    }
     switch (src) {
     case kSrcGradsSpeculative:
         return vec ? launch_update_t<kSrcGradsSpeculative, true>(a, segs, s)

@@ -60,7 +60,7 @@ struct WsHeader {
     int32_t cur;           // live ping-pong slot at the start of the step
     float bc1, bc2;        // bias corrections of the step being applied
     float clip;            // clip coefficient applied by the update
-    int32_t pad0;
+    unsigned int error;    // a bounded pipeline wait gave up (atomicOr)
     double b1p_next, b2p_next;
     double sumsq, norm;
     int64_t t_next;
@@ -86,6 +86,7 @@ struct UpdateArgs {
     float inv;                         // fp32 1/S (or 1/(S*Nd))
     float lr, beta1, beta2, eps, lr_wd;
     float one_minus_beta1, one_minus_beta2;
+    zero_step_result* result; // receives status = ZERO_ERR_TIMEOUT on a pipeline fault (may be null)
 };
 
 struct StatsArgs {
