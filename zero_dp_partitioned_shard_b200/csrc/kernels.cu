@@ -161,6 +161,42 @@ __device__ __forceinline__ void flag_nonfinite(bool bad, unsigned int* flag)
         atomicOr(flag, 1u);
 }
 
+// Walks this thread's share of a launch: the 8-element chunks of every
+// segment as one index space (segments back to back, grid-stride, so a launch
+// over many short segments keeps the whole grid busy instead of ending each
+// segment in a partial wave), then the < 8-element tail of each segment on
+// the lowest thread ids.  Without VEC every element is a scalar unit.
+template <bool VEC, typename ChunkFn, typename ElemFn>
+__device__ __forceinline__ void walk_segments(const SegList& segs, ChunkFn&& chunk, ElemFn&& elem)
+{
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    const int shift = VEC ? 3 : 0;
+    int64_t total = 0;
+    for (int s = 0; s < segs.count; ++s)
+        total += segs.seg[s].n >> shift;
+    int si = 0;
+    int64_t base = 0;
+    for (int64_t u = tid; u < total; u += nthr) {
+        while (u >= base + (segs.seg[si].n >> shift)) {
+            base += segs.seg[si].n >> shift;
+            ++si;
+        }
+        if (VEC)
+            chunk(segs.seg[si], (u - base) << 3);
+        else
+            elem(segs.seg[si], u - base);
+    }
+    if (VEC) {
+        for (int s = 0; s < segs.count; ++s) {
+            const Seg& sg = segs.seg[s];
+            const int64_t e = ((sg.n >> 3) << 3) + tid;
+            if (e < sg.n)
+                elem(sg, e);
+        }
+    }
+}
+
 __device__ __forceinline__ AdamK load_consts(const UpdateArgs& a, const WsHeader* ws, bool clip)
 {
     AdamK k;
@@ -238,7 +274,7 @@ __device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg
 }
 
 template <int SRC, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
 {
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
@@ -257,15 +293,10 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
     float* m_out = nxt ? a.exp_avg[1] : a.exp_avg[0];
     float* v_out = nxt ? a.exp_avg_sq[1] : a.exp_avg_sq[0];
 
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
     bool bad = false;
-
-    for (int si = 0; si < segs.count; ++si) {
-        const Seg& sg = segs.seg[si];
-        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
-        for (int64_t c = tid; c < n_vec; c += nthr) {
-            const int64_t e = c << 3;
+    walk_segments<VEC>(
+        segs,
+        [&](const Seg& sg, int64_t e) {
             const int64_t so = sg.s_off + e;
             float p[8], m[8], v[8], g[8];
             ld_f8(p_in + so, p);
@@ -291,11 +322,10 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             st_f8(m_out + so, m);
             st_f8(v_out + so, v);
             __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8(p));
-        }
-        // scalar elements: everything (VEC = false) or the < 8 tail
-        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr)
+        },
+        [&](const Seg& sg, int64_t e) {
             bad |= update_scalar<SRC>(a, sg, e, k, p_in, m_in, v_in, p_out, m_out, v_out);
-    }
+        });
     if (kSpec)
         flag_nonfinite(bad, &a.ws->overflow);
 }
@@ -628,18 +658,14 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
 // ---------------------------------------------------------------------------
 
 template <bool VEC, bool STASH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
 {
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
     double acc = 0.0;
     bool bad = false;
-    for (int si = 0; si < segs.count; ++si) {
-        const Seg& sg = segs.seg[si];
-        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
-        for (int64_t c = tid; c < n_vec; c += nthr) {
-            const int64_t e = c << 3;
+    walk_segments<VEC>(
+        segs,
+        [&](const Seg& sg, int64_t e) {
             float g[8];
             rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
 #pragma unroll
@@ -651,16 +677,15 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
             }
             if (STASH)
                 st_f8(a.stash + sg.s_off + e, g);
-        }
-        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr) {
+        },
+        [&](const Seg& sg, int64_t e) {
             const float g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
             bad |= !isfinite(g);
             const double d = (double)g;
             acc = __dadd_rn(acc, __dmul_rn(d, d));
             if (STASH)
                 a.stash[sg.s_off + e] = g;
-        }
-    }
+        });
     flag_nonfinite(bad, &a.ws->overflow);
 
     // fixed-pattern block reduction of the fp64 partial sums
@@ -744,20 +769,14 @@ zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_no
 template <bool VEC>
 __device__ __forceinline__ void cast_segments(const float* master, uint16_t* params, const SegList& segs)
 {
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    for (int si = 0; si < segs.count; ++si) {
-        const Seg& sg = segs.seg[si];
-        const int64_t n_vec = VEC ? (sg.n >> 3) : 0;
-        for (int64_t c = tid; c < n_vec; c += nthr) {
-            const int64_t e = c << 3;
+    walk_segments<VEC>(
+        segs,
+        [&](const Seg& sg, int64_t e) {
             float p[8];
             ld_f8(master + sg.s_off + e, p);
             __stcs(reinterpret_cast<uint4*>(params + sg.p_off + e), pack_h8(p));
-        }
-        for (int64_t e = (n_vec << 3) + tid; e < sg.n; e += nthr)
-            params[sg.p_off + e] = f2h(master[sg.s_off + e]);
-    }
+        },
+        [&](const Seg& sg, int64_t e) { params[sg.p_off + e] = f2h(master[sg.s_off + e]); });
 }
 
 template <bool VEC>
@@ -808,16 +827,33 @@ template <bool VEC>
 __global__ void __launch_bounds__(kThreads)
 zs_gather_kernel(uint16_t* dst, const __grid_constant__ GatherList g)
 {
+    // the shards' 8-element chunks as one index space (see walk_segments)
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    for (int k = 0; k < g.count; ++k) {
+    const int shift = VEC ? 3 : 0;
+    int64_t total = 0;
+    for (int k = 0; k < g.count; ++k)
+        total += g.e[k].n >> shift;
+    int k = 0;
+    int64_t base = 0;
+    for (int64_t u = tid; u < total; u += nthr) {
+        while (u >= base + (g.e[k].n >> shift)) {
+            base += g.e[k].n >> shift;
+            ++k;
+        }
         const GatherEntry& ge = g.e[k];
-        uint16_t* out = dst + ge.dst_off;
-        const int64_t n_vec = VEC ? (ge.n >> 3) : 0;
-        for (int64_t c = tid; c < n_vec; c += nthr)
-            __stcs(reinterpret_cast<uint4*>(out) + c, ld_stream(ge.src + (c << 3)));
-        for (int64_t e = (n_vec << 3) + tid; e < ge.n; e += nthr)
-            out[e] = ge.src[e];
+        if (VEC)
+            __stcs(reinterpret_cast<uint4*>(dst + ge.dst_off) + (u - base), ld_stream(ge.src + ((u - base) << 3)));
+        else
+            dst[ge.dst_off + (u - base)] = ge.src[u - base];
+    }
+    if (VEC) {
+        for (int j = 0; j < g.count; ++j) {
+            const GatherEntry& ge = g.e[j];
+            const int64_t e = ((ge.n >> 3) << 3) + tid;
+            if (e < ge.n)
+                dst[ge.dst_off + e] = ge.src[e];
+        }
     }
 }
 
@@ -888,13 +924,12 @@ static cudaError_t grid_for(K kernel, int64_t work_threads, int cap, int* blocks
     return cudaSuccess;
 }
 
+// units of work of a launch (8-element chunks when vectorised), all segments
 static int64_t seg_work(const SegList& s, bool vec)
 {
     int64_t w = 0;
-    for (int i = 0; i < s.count; ++i) {
-        const int64_t t = vec ? (s.seg[i].n + 7) >> 3 : s.seg[i].n;
-        w = t > w ? t : w;
-    }
+    for (int i = 0; i < s.count; ++i)
+        w += vec ? (s.seg[i].n + 7) >> 3 : s.seg[i].n;
     return w;
 }
 
@@ -1102,10 +1137,8 @@ cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const S
 cudaError_t launch_gather(bool vec, uint16_t* dst, const GatherList& g, cudaStream_t s)
 {
     int64_t w = 0;
-    for (int i = 0; i < g.count; ++i) {
-        const int64_t t = vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
-        w = t > w ? t : w;
-    }
+    for (int i = 0; i < g.count; ++i)
+        w += vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
     int blocks = 0;
     cudaError_t e = vec ? grid_for(zs_gather_kernel<true>, w, 0, &blocks)
                         : grid_for(zs_gather_kernel<false>, w, 0, &blocks);
