@@ -153,6 +153,15 @@ __device__ __forceinline__ float rank_sum1(const uint16_t* g, int64_t rstride, i
     return s;
 }
 
+// Programmatic dependent launch (stream-ordered, no flags): a kernel launched
+// with programmatic serialization may start while its predecessor in the
+// stream drains; griddepcontrol.wait returns once that predecessor has
+// completed and its writes are visible.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void wait_for_predecessor() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void flag_nonfinite(bool bad, unsigned int* flag)
 {
     // every lane of the warp reaches this point (grid-stride loops only)
@@ -278,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
 {
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
+    wait_for_predecessor(); // bias corrections, slot, skip and clip come from the kernels before
+    allow_dependents();
     const WsHeader* ws = a.ws;
     if (!kSpec && ws->skip)
         return; // uniform across the grid: the whole step is skipped
@@ -487,6 +498,8 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
 {
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
     constexpr int T = kPipeConsumers * EPT; // elements per tile
+    wait_for_predecessor();
+    allow_dependents();
     WsHeader* ws = a.ws;
     if (!kSpec && ws->skip)
         return; // uniform: the whole step is skipped
@@ -661,6 +674,12 @@ template <bool VEC, bool STASH>
 __global__ void __launch_bounds__(kThreads, 2)
 zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
 {
+    // The buckets of a step are independent: the next statistics launch may
+    // start as soon as this one is resident.  Each launch waits for its
+    // predecessor only before publishing its flag and partial sums, so launches
+    // overlap at their boundaries while completion stays ordered (the flag was
+    // reset by the prep kernel that heads the chain).
+    allow_dependents();
     double acc = 0.0;
     bool bad = false;
     walk_segments<VEC>(
@@ -686,6 +705,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
             if (STASH)
                 a.stash[sg.s_off + e] = g;
         });
+    wait_for_predecessor();
     flag_nonfinite(bad, &a.ws->overflow);
 
     // fixed-pattern block reduction of the fp64 partial sums
@@ -716,6 +736,8 @@ __global__ void __launch_bounds__(kFinalizeThreads)
 zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_norm,
                    zero_opt_state* st, zero_step_result* res)
 {
+    wait_for_predecessor();
+    allow_dependents();
     double acc = 0.0;
     for (int64_t i = threadIdx.x; i < n; i += kFinalizeThreads)
         acc = __dadd_rn(acc, partials[i]);
@@ -784,6 +806,7 @@ __global__ void __launch_bounds__(kThreads)
 zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int bookkeeping,
                  zero_opt_state* st, zero_step_result* res)
 {
+    wait_for_predecessor();
     const WsHeader* ws = a.ws;
     const bool fault = ws->error != 0u;
     const bool over = ws->overflow != 0u || fault;
@@ -937,6 +960,26 @@ static int64_t seg_work(const SegList& s, bool vec)
 // launchers
 // ---------------------------------------------------------------------------
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// its predecessor in the stream drains (it orders itself with
+// griddepcontrol.wait).  Used for the kernels after the first of a step.
+template <typename... Params, typename... Args>
+static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                                     cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 cudaError_t launch_opt_init(zero_opt_state* st, cudaStream_t s)
 {
     zs_opt_init_kernel<<<1, 1, 0, s>>>(st);
@@ -959,9 +1002,9 @@ static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, cud
     cudaError_t e = grid_for(zs_update_kernel<SRC, VEC>, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    zs_update_kernel<SRC, VEC><<<blocks, kThreads, 0, s>>>(a, segs);
+    e = launch_overlapped(zs_update_kernel<SRC, VEC>, blocks, kThreads, 0, s, a, segs);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 // Shape of the pipelined update for a given source: elements per consumer
@@ -1024,9 +1067,9 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
     int64_t grid = (int64_t)sms * ps.ctas_per_sm;
     grid = tiles < grid ? tiles : grid;
     grid = grid < 1 ? 1 : grid;
-    kernel<<<(unsigned)grid, kPipeThreads, ps.smem, s>>>(a, segs, ps.stages);
+    e = launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 template <int SRC>
@@ -1081,9 +1124,10 @@ int stats_blocks(bool vec, const SegList& segs)
 template <bool VEC, bool STASH>
 static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, cudaStream_t s)
 {
-    zs_stats_kernel<VEC, STASH><<<stats_blocks(VEC, segs), kThreads, 0, s>>>(a, segs);
+    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH>, stats_blocks(VEC, segs), kThreads, 0, s,
+                                            a, segs);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
@@ -1097,9 +1141,10 @@ cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cuda
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, float max_norm,
                             zero_opt_state* st, zero_step_result* res, cudaStream_t s)
 {
-    zs_finalize_kernel<<<1, kFinalizeThreads, 0, s>>>(ws, partials, n, max_norm, st, res);
+    const cudaError_t e = launch_overlapped(zs_finalize_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n,
+                                            max_norm, st, res);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
@@ -1110,12 +1155,11 @@ cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bo
                         : grid_for(zs_commit_kernel<false>, seg_work(segs, false), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    if (vec)
-        zs_commit_kernel<true><<<blocks, kThreads, 0, s>>>(a, segs, bookkeeping ? 1 : 0, st, res);
-    else
-        zs_commit_kernel<false><<<blocks, kThreads, 0, s>>>(a, segs, bookkeeping ? 1 : 0, st, res);
+    e = vec ? launch_overlapped(zs_commit_kernel<true>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res)
+            : launch_overlapped(zs_commit_kernel<false>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st,
+                                res);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
