@@ -335,6 +335,15 @@ ZERO_API const char* zero_strerror(zero_status status);
 ZERO_API const char* zero_last_error(void);
 /* Number of kernels this library has launched in this process. */
 ZERO_API uint64_t zero_launch_count(void);
+/* Budget, in SM clock cycles, of each bounded wait inside the pipelined
+ * update kernel (default 2^31, about a second).  A wait that exceeds it makes
+ * the step report status ZERO_ERR_TIMEOUT instead of hanging.  A negative
+ * value makes every such wait expire at once (a test hook for that path: the
+ * kernel then copies and updates nothing).  The final wait for the kernel's
+ * own copies in flight always keeps the default budget.  0 restores the
+ * default.  Returns the previous value.  Process-wide; affects steps
+ * enqueued afterwards. */
+ZERO_API int64_t zero_set_wait_budget(int64_t cycles);
 
 #ifdef __cplusplus
 }

@@ -242,3 +242,11 @@ def test_strerror_names_every_status():
     for s in range(7):
         assert B.zero_strerror(s) and "unknown" not in B.zero_strerror(s)
     assert "unknown" in B.zero_strerror(99)
+
+
+def test_wait_budget_hook_round_trips():
+    default = B.zero_set_wait_budget(12345)
+    assert default == 1 << 31
+    assert B.zero_set_wait_budget(-1) == 12345
+    assert B.zero_set_wait_budget(0) == -1
+    assert B.zero_set_wait_budget(0) == 1 << 31

@@ -124,6 +124,7 @@ SIGNATURES = {
     "zero_strerror": (C.c_char_p, [_S]),
     "zero_last_error": (C.c_char_p, []),
     "zero_launch_count": (C.c_uint64, []),
+    "zero_set_wait_budget": (C.c_int64, [C.c_int64]),
 }
 
 
@@ -254,6 +255,12 @@ def zero_last_error() -> str:
 
 def zero_launch_count() -> int:
     return lib().zero_launch_count()
+
+
+def zero_set_wait_budget(cycles: int) -> int:
+    """Sets the per-wait cycle budget of the pipelined update (0 = default, < 0 =
+    expire at once); returns the previous value."""
+    return lib().zero_set_wait_budget(cycles)
 
 
 # ---------------------------------------------------------------------------

@@ -245,6 +245,7 @@ zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
     u.params = static_cast<uint16_t*>(a.params);
     u.ws = ws;
     u.result = res;
+    u.wait_budget = zs::wait_budget_cycles();
     u.nd = p.nd;
     double scale = (double)h.loss_scale;
     if (h.average_over_nd)

@@ -357,7 +357,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
 constexpr int kPipeConsumerWarps = 8;
 constexpr int kPipeConsumers = kPipeConsumerWarps * 32;
 constexpr int kPipeThreads = kPipeConsumers + 32; // + the producer warp
-constexpr long long kWaitBudgetCycles = 1ll << 31; // ~1 s: far beyond any memory latency
+constexpr long long kDrainBudgetCycles = 1ll << 31; // ~1 s: far beyond any memory latency
 constexpr int kPipeHeaderBytes = 1024;           // mbarriers + tile table, before the ring
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p)
@@ -393,14 +393,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase of the given parity; false if the budget ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+// Wait for the phase of the given parity; false if `budget` cycles ran out
+// (a negative budget expires at once).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long budget)
 {
+    if (budget < 0)
+        return false;
     if (mbar_test(bar, parity))
         return true;
     const long long t0 = clock64();
     while (!mbar_test(bar, parity))
-        if (clock64() - t0 > kWaitBudgetCycles)
+        if (clock64() - t0 > budget)
             return false;
     return true;
 }
@@ -549,7 +552,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
             const int st = it % stages;
             bool ok = true;
             if (lane == 0)
-                ok = mbar_wait(&empty[st], ((it / stages) & 1) ^ 1);
+                ok = mbar_wait(&empty[st], ((it / stages) & 1) ^ 1, a.wait_budget);
             if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 failed = true;
                 break;
@@ -582,7 +585,8 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
             const int issued = it;
             for (int st = 0; st < stages && st < issued; ++st) {
                 const int last = issued - 1 - ((issued - 1 - st) % stages); // last use of stage st
-                if (!mbar_wait(&full[st], (last / stages) & 1))
+                const long long drain = a.wait_budget > kDrainBudgetCycles ? a.wait_budget : kDrainBudgetCycles;
+                if (!mbar_wait(&full[st], (last / stages) & 1, drain))
                     failed = true;
             }
         }
@@ -594,7 +598,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
         int it = 0;
         for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
             const int st = it % stages;
-            const bool ok = mbar_wait(&full[st], (it / stages) & 1);
+            const bool ok = mbar_wait(&full[st], (it / stages) & 1, a.wait_budget);
             if (!__all_sync(0xffffffffu, ok)) {
                 failed = true;
                 break;

@@ -16,6 +16,10 @@ namespace zs {
 
 static thread_local char g_last_error[512] = "";
 static std::atomic<uint64_t> g_launches{0};
+constexpr int64_t kDefaultWaitBudget = 1ll << 31; // about a second at B200 clocks
+static std::atomic<int64_t> g_wait_budget{kDefaultWaitBudget};
+
+long long wait_budget_cycles() { return (long long)g_wait_budget.load(std::memory_order_relaxed); }
 
 zero_status fail(zero_status s, const char* fmt, ...)
 {
@@ -55,6 +59,11 @@ const char* zero_strerror(zero_status s)
 const char* zero_last_error(void) { return zs::g_last_error; }
 
 uint64_t zero_launch_count(void) { return zs::g_launches.load(std::memory_order_relaxed); }
+
+int64_t zero_set_wait_budget(int64_t cycles)
+{
+    return zs::g_wait_budget.exchange(cycles ? cycles : zs::kDefaultWaitBudget);
+}
 
 // Shard length: the smallest multiple of A whose Nd copies cover Psi.
 zero_status zero_plan(const zero_plan_desc* d, zero_plan_t** out)

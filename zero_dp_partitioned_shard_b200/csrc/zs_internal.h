@@ -28,6 +28,7 @@ namespace zs {
 zero_status fail(zero_status s, const char* fmt, ...);
 void clear_error();
 void count_launches(uint64_t n);
+long long wait_budget_cycles();  // current budget of a bounded pipeline wait
 
 // ---- launch geometry ------------------------------------------------------------
 constexpr int kThreads = 256;          // threads per block of the streaming kernels
@@ -87,6 +88,7 @@ struct UpdateArgs {
     float lr, beta1, beta2, eps, lr_wd;
     float one_minus_beta1, one_minus_beta2;
     zero_step_result* result; // receives status = ZERO_ERR_TIMEOUT on a pipeline fault (may be null)
+    long long wait_budget;    // cycles per bounded pipeline wait
 };
 
 struct StatsArgs {
