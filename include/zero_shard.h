@@ -280,6 +280,32 @@ ZERO_API zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hp
 ZERO_API zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
                             const zero_step_args* args, void* stream);
 
+/* ---- split step: one owner per process -------------------------------------- */
+/* When each owner runs in its own process (one GPU each), a step's global
+ * decisions -- skip on a non-finite gradient anywhere, the global clip norm --
+ * need every owner's gradient.  zero_shard_step_begin and _end split the step
+ * around one sum-all-reduce of a 16-byte "vote" that the library keeps in the
+ * workspace at byte offset ZERO_VOTE_OFFSET: two fp64 values, {this call's
+ * sum of squares of the unscaled reduced gradient (0 in SPECULATIVE mode),
+ * 1 if this call saw a non-finite gradient else 0}.  The caller adds the
+ * votes of all processes (e.g. an NCCL fp64 sum over the group, in place on
+ * the stream between the two calls); any non-zero second value then skips
+ * the step everywhere, and the summed first value gives the global norm.
+ *   SPECULATIVE: begin = fused update into the spare slot + vote; end =
+ *     commit (or re-cast on skip).  TWO_PASS / STASH: begin = statistics
+ *     pass + vote; end = decision + in-place update.
+ * begin + end with no reduction in between equal zero_shard_step over the
+ * call's owners; arguments, workspace and errors are those of
+ * zero_shard_step, and both calls must receive the same arguments.  The
+ * exchange of gradient slices before begin (each owner gathers the Nd
+ * contributions to its shard: the reduce-scatter's input) and the
+ * all-gather of the fp16 shards after end are the caller's collectives. */
+#define ZERO_VOTE_OFFSET 128
+ZERO_API zero_status zero_shard_step_begin(const zero_plan_t* plan, const zero_hparams* hp,
+                                           const zero_step_args* args, void* stream);
+ZERO_API zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hparams* hp,
+                                         const zero_step_args* args, void* stream);
+
 /* Size of the device scratch array that zero_shard_step_static_scratch uses
  * (1 MiB on every GPU that loads the library, kept until the process exits). */
 #define ZERO_STATIC_SCRATCH_BYTES (1 << 20)

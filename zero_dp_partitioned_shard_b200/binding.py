@@ -34,6 +34,7 @@ ZERO_GRADS_FULL = 0
 ZERO_GRADS_PER_OWNER = 1
 
 ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
+ZERO_VOTE_OFFSET = 128               # byte offset of the split step's fp64[2] vote in the workspace
 
 OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (40 bytes used)
 RESULT_BYTES = 64      # device allocation for zero_step_result (40 bytes used)
@@ -118,6 +119,8 @@ SIGNATURES = {
     "zero_workspace_bytes": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), C.POINTER(C.c_size_t)]),
     "zero_shard_step": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_static_scratch": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
+    "zero_shard_step_begin": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
+    "zero_shard_step_end": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, _P]),
     "zero_abi_version": (C.c_int32, []),
@@ -227,6 +230,16 @@ def zero_shard_step_static_scratch(plan: int, hp: HParams, args: StepArgs, strea
     """zero_shard_step with the library's static device scratch (args.workspace ignored)."""
     _check(lib().zero_shard_step_static_scratch(plan, C.byref(hp), C.byref(args), stream),
            "zero_shard_step_static_scratch")
+
+
+def zero_shard_step_begin(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
+    """First half of a split step: ends with this call's vote at workspace + ZERO_VOTE_OFFSET."""
+    _check(lib().zero_shard_step_begin(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step_begin")
+
+
+def zero_shard_step_end(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
+    """Second half of a split step, after the votes of all owners were summed in place."""
+    _check(lib().zero_shard_step_end(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step_end")
 
 
 def zero_gather_params(plan: int, shard_ptrs, params_full: int, stream: int = 0) -> None:

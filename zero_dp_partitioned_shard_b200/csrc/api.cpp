@@ -207,8 +207,12 @@ zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hparams* hp
     return ZERO_OK;
 }
 
-zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
-                            const zero_step_args* args, void* stream)
+// The step's kernel sequence.  PHASE_ALL is zero_shard_step; PHASE_BEGIN and
+// PHASE_END are its two halves around the caller's reduction of the vote.
+enum StepPhase { PHASE_ALL, PHASE_BEGIN, PHASE_END };
+
+static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, const zero_step_args* args,
+                            void* stream, StepPhase phase)
 {
     zs::clear_error();
     zero_status s = validate(plan, hp, args);
@@ -260,52 +264,93 @@ zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
     u.one_minus_beta1 = 1.0f - h.beta1;
     u.one_minus_beta2 = 1.0f - h.beta2;
 
-    cudaError_t e = zs::launch_prep(st, ws, h.beta1, h.beta2, str);
-    if (e != cudaSuccess)
+    const bool spec = h.mode == ZERO_MODE_SPECULATIVE;
+    const bool first_half = phase != PHASE_END;
+    const bool second_half = phase != PHASE_BEGIN;
+    cudaError_t e;
+    if (first_half && (e = zs::launch_prep(st, ws, h.beta1, h.beta2, str)) != cudaSuccess)
         return cuda_fail(e, "prep launch");
 
-    if (h.mode == ZERO_MODE_SPECULATIVE) {
-        if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
-            return cuda_fail(e, "timing event");
-        for (const auto& b : lp.buckets)
-            for (const auto& l : b)
-                if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, str)) != cudaSuccess)
-                    return cuda_fail(e, "update launch");
-        if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
-            return cuda_fail(e, "timing event");
-        for (size_t i = 0; i < lp.whole.size(); ++i)
-            if ((e = zs::launch_commit(lp.vec, u, lp.whole[i], i == 0, st, res, str)) != cudaSuccess)
-                return cuda_fail(e, "commit launch");
+    if (spec) {
+        if (first_half) {
+            if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+                return cuda_fail(e, "timing event");
+            for (const auto& b : lp.buckets)
+                for (const auto& l : b)
+                    if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, str)) != cudaSuccess)
+                        return cuda_fail(e, "update launch");
+            if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+                return cuda_fail(e, "timing event");
+            if (phase == PHASE_BEGIN && (e = zs::launch_vote_local(ws, partials, 0, str)) != cudaSuccess)
+                return cuda_fail(e, "vote launch");
+        }
+        if (second_half) {
+            if (phase == PHASE_END &&
+                (e = zs::launch_vote_apply(ws, true, h.max_grad_norm, st, res, str)) != cudaSuccess)
+                return cuda_fail(e, "vote launch");
+            for (size_t i = 0; i < lp.whole.size(); ++i)
+                if ((e = zs::launch_commit(lp.vec, u, lp.whole[i], i == 0, st, res, str)) != cudaSuccess)
+                    return cuda_fail(e, "commit launch");
+        }
         return ZERO_OK;
     }
 
-    // pre-pass modes: statistics bucket by bucket, finalize, in-place update
-    zs::StatsArgs sa;
-    sa.grads = u.grads;
-    sa.stash = h.mode == ZERO_MODE_STASH ? a.grad_stash : nullptr;
-    sa.ws = ws;
-    sa.nd = p.nd;
-    sa.inv = u.inv;
-    int64_t n_partials = 0;
-    for (const auto& b : lp.buckets) {
-        for (const auto& l : b) {
-            sa.partials = partials + n_partials;
-            if ((e = zs::launch_stats(lp.vec, sa, l, str)) != cudaSuccess)
-                return cuda_fail(e, "statistics launch");
-            n_partials += zs::stats_blocks(lp.vec, l);
+    // pre-pass modes: statistics bucket by bucket, decision, in-place update
+    if (first_half) {
+        zs::StatsArgs sa;
+        sa.grads = u.grads;
+        sa.stash = h.mode == ZERO_MODE_STASH ? a.grad_stash : nullptr;
+        sa.ws = ws;
+        sa.nd = p.nd;
+        sa.inv = u.inv;
+        int64_t n_partials = 0;
+        for (const auto& b : lp.buckets) {
+            for (const auto& l : b) {
+                sa.partials = partials + n_partials;
+                if ((e = zs::launch_stats(lp.vec, sa, l, str)) != cudaSuccess)
+                    return cuda_fail(e, "statistics launch");
+                n_partials += zs::stats_blocks(lp.vec, l);
+            }
+        }
+        if (phase == PHASE_ALL) {
+            if ((e = zs::launch_finalize(ws, partials, n_partials, h.max_grad_norm, st, res, str)) != cudaSuccess)
+                return cuda_fail(e, "finalize launch");
+        } else if ((e = zs::launch_vote_local(ws, partials, n_partials, str)) != cudaSuccess) {
+            return cuda_fail(e, "vote launch");
         }
     }
-    if ((e = zs::launch_finalize(ws, partials, n_partials, h.max_grad_norm, st, res, str)) != cudaSuccess)
-        return cuda_fail(e, "finalize launch");
-    const int src = h.mode == ZERO_MODE_STASH ? zs::kSrcStash : zs::kSrcGradsInPlace;
-    if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
-        return cuda_fail(e, "timing event");
-    for (const auto& l : lp.whole)
-        if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, str)) != cudaSuccess)
-            return cuda_fail(e, "update launch");
-    if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
-        return cuda_fail(e, "timing event");
+    if (second_half) {
+        if (phase == PHASE_END &&
+            (e = zs::launch_vote_apply(ws, false, h.max_grad_norm, st, res, str)) != cudaSuccess)
+            return cuda_fail(e, "vote launch");
+        const int src = h.mode == ZERO_MODE_STASH ? zs::kSrcStash : zs::kSrcGradsInPlace;
+        if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+            return cuda_fail(e, "timing event");
+        for (const auto& l : lp.whole)
+            if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, str)) != cudaSuccess)
+                return cuda_fail(e, "update launch");
+        if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+            return cuda_fail(e, "timing event");
+    }
     return ZERO_OK;
+}
+
+zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
+                            const zero_step_args* args, void* stream)
+{
+    return run_step(plan, hp, args, stream, PHASE_ALL);
+}
+
+zero_status zero_shard_step_begin(const zero_plan_t* plan, const zero_hparams* hp,
+                                  const zero_step_args* args, void* stream)
+{
+    return run_step(plan, hp, args, stream, PHASE_BEGIN);
+}
+
+zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hparams* hp,
+                                const zero_step_args* args, void* stream)
+{
+    return run_step(plan, hp, args, stream, PHASE_END);
 }
 
 zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard_ptrs,

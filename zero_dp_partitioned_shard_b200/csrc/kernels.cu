@@ -736,12 +736,9 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
 
 constexpr int kFinalizeThreads = 1024;
 
-__global__ void __launch_bounds__(kFinalizeThreads)
-zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_norm,
-                   zero_opt_state* st, zero_step_result* res)
+__device__ __forceinline__ double block_sum_partials(const double* partials, int64_t n)
 {
-    wait_for_predecessor();
-    allow_dependents();
+    // fixed order: thread i sums partials i, i + 1024, ... ; then a fixed tree
     double acc = 0.0;
     for (int64_t i = threadIdx.x; i < n; i += kFinalizeThreads)
         acc = __dadd_rn(acc, partials[i]);
@@ -752,22 +749,28 @@ zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_no
     if ((threadIdx.x & 31) == 0)
         warp_sum[threadIdx.x >> 5] = acc;
     __syncthreads();
-    if (threadIdx.x >= 32)
-        return;
-    double w = warp_sum[threadIdx.x];
+    double w = 0.0;
+    if (threadIdx.x < 32) {
+        w = warp_sum[threadIdx.x];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        w = __dadd_rn(w, __shfl_down_sync(0xffffffffu, w, off));
-    if (threadIdx.x != 0)
-        return;
-    const bool skip = ws->overflow != 0u;
-    const double norm = __dsqrt_rn(w);
+        for (int off = 16; off > 0; off >>= 1)
+            w = __dadd_rn(w, __shfl_down_sync(0xffffffffu, w, off));
+    }
+    return w; // valid in thread 0
+}
+
+// The step's global decision from the gradient's sum of squares and the
+// overflow vote: norm, clip coefficient, skip, optimizer bookkeeping, result.
+__device__ __forceinline__ void decide_step(WsHeader* ws, double sumsq, bool skip, float max_norm,
+                                            zero_opt_state* st, zero_step_result* res)
+{
+    const double norm = __dsqrt_rn(sumsq);
     float clip = 1.0f;
     if (!skip && max_norm > 0.0f && norm > (double)max_norm)
         clip = __double2float_rn(__ddiv_rn((double)max_norm, norm));
     ws->skip = skip ? 1 : 0;
     ws->clip = clip;
-    ws->sumsq = w;
+    ws->sumsq = sumsq;
     ws->norm = norm;
     if (!skip) {
         st->t = ws->t_next;
@@ -785,6 +788,47 @@ zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_no
         res->status = ZERO_OK;
         res->reserved = 0;
     }
+}
+
+__global__ void __launch_bounds__(kFinalizeThreads)
+zs_finalize_kernel(WsHeader* ws, const double* partials, int64_t n, float max_norm,
+                   zero_opt_state* st, zero_step_result* res)
+{
+    wait_for_predecessor();
+    allow_dependents();
+    const double w = block_sum_partials(partials, n);
+    if (threadIdx.x == 0)
+        decide_step(ws, w, ws->overflow != 0u, max_norm, st, res);
+}
+
+// Split step, first half's end: this call's share of the global vote --
+// its sum of squares (0 without a statistics pass) and whether it saw a
+// non-finite gradient -- as two fp64 values that callers running one owner
+// per process add up across processes (one sum-all-reduce of 16 bytes).
+__global__ void __launch_bounds__(kFinalizeThreads)
+zs_vote_local_kernel(WsHeader* ws, const double* partials, int64_t n)
+{
+    wait_for_predecessor();
+    allow_dependents();
+    const double w = block_sum_partials(partials, n);
+    if (threadIdx.x == 0) {
+        ws->vote[0] = w;
+        ws->vote[1] = ws->overflow != 0u ? 1.0 : 0.0;
+    }
+}
+
+// Split step, second half's start: the (now global) vote decides the step.
+// Speculative: only the overflow flag, which the commit kernel then applies.
+__global__ void zs_vote_apply_kernel(WsHeader* ws, int speculative, float max_norm, zero_opt_state* st,
+                                     zero_step_result* res)
+{
+    wait_for_predecessor();
+    allow_dependents();
+    const bool skip = ws->vote[1] != 0.0;
+    if (speculative)
+        ws->overflow = skip ? 1u : 0u;
+    else
+        decide_step(ws, ws->vote[0], skip, max_norm, st, res);
 }
 
 // ---------------------------------------------------------------------------
@@ -1149,6 +1193,22 @@ cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, flo
                                             max_norm, st, res);
     count_launches(1);
     return e;
+}
+
+cudaError_t launch_vote_local(WsHeader* ws, const double* partials, int64_t n, cudaStream_t s)
+{
+    const cudaError_t e = launch_overlapped(zs_vote_local_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n);
+    count_launches(1);
+    return e;
+}
+
+cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, zero_opt_state* st,
+                              zero_step_result* res, cudaStream_t s)
+{
+    // an ordinary launch: the caller's all-reduce of the vote comes before it
+    zs_vote_apply_kernel<<<1, 1, 0, s>>>(ws, speculative ? 1 : 0, max_norm, st, res);
+    count_launches(1);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,

@@ -65,8 +65,11 @@ struct WsHeader {
     double b1p_next, b2p_next;
     double sumsq, norm;
     int64_t t_next;
+    unsigned char pad1[ZERO_VOTE_OFFSET - 72];
+    double vote[2]; // split step: {sum of squares, non-finite seen}, at ZERO_VOTE_OFFSET
 };
 static_assert(sizeof(WsHeader) <= kHeaderBytes, "workspace header too large");
+static_assert(offsetof(WsHeader, vote) == ZERO_VOTE_OFFSET, "vote must sit at ZERO_VOTE_OFFSET");
 
 // Source of the reduced gradient in the update kernel.
 enum UpdateSrc : int {
@@ -124,6 +127,9 @@ cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cuda
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n_partials,
                             float max_grad_norm, zero_opt_state* st, zero_step_result* res,
                             cudaStream_t s);
+cudaError_t launch_vote_local(WsHeader* ws, const double* partials, int64_t n, cudaStream_t s);
+cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, zero_opt_state* st,
+                              zero_step_result* res, cudaStream_t s);
 cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
                           zero_opt_state* st, zero_step_result* res, cudaStream_t s);
 cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
