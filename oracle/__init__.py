@@ -51,7 +51,9 @@ class HParams(C.Structure):
 
 
 class OptState(C.Structure):
-    _fields_ = [("t", C.c_int64), ("beta1_pow", C.c_double), ("beta2_pow", C.c_double)]
+    _fields_ = [("t", C.c_int64), ("beta1_pow", C.c_double), ("beta2_pow", C.c_double),
+                ("loss_scale", C.c_float), ("good_steps", C.c_int32), ("growth_factor", C.c_float),
+                ("backoff_factor", C.c_float), ("growth_interval", C.c_int32), ("pad_", C.c_int32)]
 
 
 class StepInfo(C.Structure):
@@ -257,11 +259,24 @@ class Opt:
     t: int = 0
     beta1_pow: float = 1.0
     beta2_pow: float = 1.0
+    loss_scale: float = 0.0        # > 0: dynamic loss scaling with this current scale
+    good_steps: int = 0
+    growth_factor: float = 2.0
+    backoff_factor: float = 0.5
+    growth_interval: int = 2000
+
+    def _c(self) -> OptState:
+        return OptState(self.t, self.beta1_pow, self.beta2_pow, self.loss_scale, self.good_steps,
+                        self.growth_factor, self.backoff_factor, self.growth_interval, 0)
+
+    def _update(self, o: OptState) -> None:
+        self.t, self.beta1_pow, self.beta2_pow = o.t, o.beta1_pow, o.beta2_pow
+        self.loss_scale, self.good_steps = o.loss_scale, o.good_steps
 
 
 def bias_corrections(hp: HP, opt: Opt):
     """(beta1^(t+1), beta2^(t+1), fp32 bc1, fp32 bc2) for the next step."""
-    h, o = hp._c(), OptState(opt.t, opt.beta1_pow, opt.beta2_pow)
+    h, o = hp._c(), opt._c()
     b1, b2, c1, c2 = C.c_double(), C.c_double(), C.c_float(), C.c_float()
     lib().oracle_bias_corrections(C.byref(h), C.byref(o), C.byref(b1), C.byref(b2),
                                   C.byref(c1), C.byref(c2))
@@ -282,7 +297,7 @@ def step(G: np.ndarray, master: np.ndarray, exp_avg: np.ndarray, exp_avg_sq: np.
                   (params, np.uint16)):
         assert a.dtype == dt and a.flags["C_CONTIGUOUS"] and a.size == psi
     h = hp._c()
-    o = OptState(opt.t, opt.beta1_pow, opt.beta2_pow)
+    o = opt._c()
     info = StepInfo()
     rc = lib().oracle_step(_ptr(G), G.shape[1], G.shape[0], psi, _ptr(master), _ptr(exp_avg),
                            _ptr(exp_avg_sq), _ptr(params), C.byref(h), C.byref(o),
@@ -291,7 +306,7 @@ def step(G: np.ndarray, master: np.ndarray, exp_avg: np.ndarray, exp_avg_sq: np.
                            threads, C.byref(info))
     if rc != 0:
         raise ValueError("oracle_step rejected its arguments")
-    opt.t, opt.beta1_pow, opt.beta2_pow = o.t, o.beta1_pow, o.beta2_pow
+    opt._update(o)
     return {name: getattr(info, name) for name, _ in StepInfo._fields_}
 
 

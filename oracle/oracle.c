@@ -395,6 +395,19 @@ typedef struct {
     int64_t t;        /* steps applied so far */
     double beta1_pow; /* beta1^t, fp64 running product, starts at 1 */
     double beta2_pow;
+    /* Dynamic loss scaling (Micikevicius et al. 2018, "Mixed Precision
+     * Training", section 3.2; the pages cite that paper only as background):
+     * in use when loss_scale > 0, which then replaces the static S of the
+     * hyper-parameters.  A skipped step multiplies the scale by
+     * backoff_factor; growth_interval consecutive applied steps multiply it by
+     * growth_factor.  good_steps counts the applied steps since the last
+     * change. */
+    float loss_scale;
+    int32_t good_steps;
+    float growth_factor;
+    float backoff_factor;
+    int32_t growth_interval;
+    int32_t pad_;
 } oracle_opt_state;
 
 typedef struct {
@@ -429,12 +442,38 @@ static void comp_add(comp_sum* a, double t)
 }
 
 /* Unscale factor: fp32 reciprocal of S (times 1/Nd when averaging). */
-static float unscale_factor(const oracle_hparams* hp, int32_t nd)
+static float unscale_factor_of(float loss_scale, int32_t average, int32_t nd)
 {
-    double d = (double)hp->loss_scale;
-    if (hp->average_over_nd)
+    double d = (double)loss_scale;
+    if (average)
         d *= (double)nd;
     return (float)(1.0 / d);
+}
+
+static float unscale_factor(const oracle_hparams* hp, int32_t nd)
+{
+    return unscale_factor_of(hp->loss_scale, hp->average_over_nd, nd);
+}
+
+/* The loss scale a step divides by: the dynamic one when in use. */
+static float step_loss_scale(const oracle_hparams* hp, const oracle_opt_state* st)
+{
+    return st->loss_scale > 0.0f ? st->loss_scale : hp->loss_scale;
+}
+
+/* Dynamic loss scaling after a step: back off on a skip, grow after
+ * growth_interval consecutive applied steps (fp32 products). */
+static void advance_loss_scale(oracle_opt_state* st, int32_t skipped)
+{
+    if (!(st->loss_scale > 0.0f))
+        return;
+    if (skipped) {
+        st->loss_scale = st->loss_scale * st->backoff_factor;
+        st->good_steps = 0;
+    } else if (++st->good_steps >= st->growth_interval) {
+        st->loss_scale = st->loss_scale * st->growth_factor;
+        st->good_steps = 0;
+    }
 }
 
 /* Mixed-precision Adam/AdamW on one element (Kingma & Ba 2015, Alg. 1;
@@ -525,7 +564,7 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
     float* g = (float*)malloc((size_t)psi * sizeof(float));
     if (!g)
         return -1;
-    const float inv = unscale_factor(hp, nd);
+    const float inv = unscale_factor_of(step_loss_scale(hp, st), hp->average_over_nd, nd);
 
     /* 1. reduce-scatter sum (every owner's slice) and unscale */
 #pragma omp parallel for num_threads(threads > 0 ? threads : 1) if (threads > 1) schedule(static)
@@ -546,6 +585,7 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
         info->clip_coef = 1.0f;
         info->grad_norm = NAN;
         info->sumsq = NAN;
+        advance_loss_scale(st, 1);
         free(g);
         return 0;
     }
@@ -581,6 +621,7 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
     st->t += 1;
     st->beta1_pow = b1p;
     st->beta2_pow = b2p;
+    advance_loss_scale(st, 0);
     info->clip_coef = clip;
     info->sumsq = sumsq;
     info->grad_norm = norm;

@@ -270,3 +270,47 @@ def test_threads_do_not_change_results():
         outs.append((master, m, v, P))
     for a, b in zip(*outs):
         assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_dynamic_loss_scale_state_machine():
+    """Dynamic loss scaling (Micikevicius et al. 2018, sec. 3.2; the pages
+    cite the paper as background only): halve on a skipped step, double after
+    growth_interval consecutive applied steps, counting restarts on change."""
+    nd, n, S0 = 2, 256, 2.0 ** 16
+    G_ok = synth.grads_f16(nd, n, seed=71, std=1e-3, scale=S0)
+    G_bad = G_ok.copy()
+    G_bad[1, 7] = 0x7C00
+    hp = oracle.HP(loss_scale=1.0)   # ignored while the dynamic scale is in use
+    opt = oracle.Opt(loss_scale=S0, growth_interval=3, growth_factor=2.0, backoff_factor=0.5)
+    master = synth.normal_f32(n, seed=72, std=0.02)
+    m, v, P = np.zeros(n, F32), np.zeros(n, F32), np.zeros(n, np.uint16)
+    plan = ["ok", "ok", "ok", "ok", "ok", "bad", "ok", "bad", "bad", "ok", "ok", "ok"]
+    want = [(S0, 1), (S0, 2), (2 * S0, 0), (2 * S0, 1), (2 * S0, 2), (S0, 0), (S0, 1),
+            (S0 / 2, 0), (S0 / 4, 0), (S0 / 4, 1), (S0 / 4, 2), (S0 / 2, 0)]
+    for kind, (s_after, good_after) in zip(plan, want):
+        info = oracle.step(G_bad if kind == "bad" else G_ok, master, m, v, P, hp, opt)
+        assert info["overflow"] == (kind == "bad")
+        assert (opt.loss_scale, opt.good_steps) == (s_after, good_after)
+    assert opt.t == plan.count("ok")
+
+
+def test_dynamic_scale_replaces_the_static_one():
+    nd, n, S = 4, 1000, 2.0 ** 10
+    G = synth.grads_f16(nd, n, seed=73, std=1e-3, scale=S)
+    outs = []
+    for opt, hp in ((oracle.Opt(loss_scale=S), oracle.HP(loss_scale=7.0)),
+                    (oracle.Opt(), oracle.HP(loss_scale=S))):
+        master = synth.normal_f32(n, seed=74, std=0.02)
+        m, v, P = np.zeros(n, F32), np.zeros(n, F32), np.zeros(n, np.uint16)
+        oracle.step(G, master, m, v, P, hp, opt)
+        outs.append((master, m, v, P))
+    for a, b in zip(*outs):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_static_scale_leaves_the_scale_state_alone():
+    G = synth.grads_f16(2, 100, seed=75, std=1e-3, scale=8.0)
+    opt = oracle.Opt()
+    oracle.step(G, synth.normal_f32(100, seed=1, std=0.02), np.zeros(100, F32), np.zeros(100, F32),
+                np.zeros(100, np.uint16), oracle.HP(loss_scale=8.0), opt)
+    assert (opt.loss_scale, opt.good_steps, opt.t) == (0.0, 0, 1)
