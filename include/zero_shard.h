@@ -23,7 +23,8 @@
  *
  * Arithmetic (the pages give no update equations; textbook readings):
  *   s_i  = c_0,i + c_1,i + ... + c_{Nd-1},i      fp32, left to right by rank
- *   g_i  = s_i * (fp32)(1/S)      [(fp32)(1/(S*Nd)) when averaging]
+ *   g_i  = s_i * (fp32)(1/S)      [(fp32)(1/(S*Nd)) when averaging; S is the
+ *          dynamic loss scale of zero_opt_state when one is in use]
  *   skip the whole step if any g_i (i < Psi, pads excluded) is not finite
  *   norm = sqrt(sum_i (double)g_i^2); c = max/norm if norm > max else 1
  *   g^_i = g_i * c
@@ -61,7 +62,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 2
+#define ZERO_SHARD_ABI_VERSION 3
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -191,7 +192,19 @@ typedef struct zero_opt_state {
     int64_t skipped;  /* steps skipped on overflow */
     int32_t cur;      /* SPECULATIVE: ping-pong slot (0/1) holding the live state */
     int32_t reserved;
-} zero_opt_state;
+    /* Dynamic loss scaling (mixed-precision training, Micikevicius et al.
+     * 2018, section 3.2), in use when loss_scale > 0: it then replaces
+     * zero_hparams.loss_scale; a skipped step multiplies it by
+     * backoff_factor, growth_interval consecutive applied steps multiply it
+     * by growth_factor, and good_steps counts the applied steps since the
+     * last change.  zero_opt_state_init leaves it off (loss_scale = 0). */
+    float loss_scale;
+    int32_t good_steps;
+    float growth_factor;
+    float backoff_factor;
+    int32_t growth_interval;
+    int32_t reserved2;
+} zero_opt_state; /* 64 bytes */
 
 /* Per-call outcome, written to device memory when args->result != NULL. */
 typedef struct zero_step_result {
@@ -205,7 +218,7 @@ typedef struct zero_step_result {
                           kernel gave up (a fault, never expected): SPECULATIVE
                           then keeps the previous state as on overflow; in
                           TWO_PASS / STASH the update is incomplete */
-    int32_t reserved;
+    float loss_scale;  /* dynamic loss scale for the next step (0: static scaling) */
 } zero_step_result;
 
 /* ---- the step ---------------------------------------------------------------------- */
@@ -254,9 +267,14 @@ typedef struct zero_step_args {
     void* timing_events[2];
 } zero_step_args;
 
-/* Writes {t = 0, beta1_pow = beta2_pow = 1, skipped = 0, cur = 0} into the
- * device zero_opt_state at opt_state, on stream. */
+/* Writes {t = 0, beta1_pow = beta2_pow = 1, skipped = 0, cur = 0, static
+ * loss scaling} into the device zero_opt_state at opt_state, on stream. */
 ZERO_API zero_status zero_opt_state_init(void* opt_state, void* stream);
+/* The same with dynamic loss scaling switched on, starting at initial_scale.
+ * Errors: INVALID_ARG unless initial_scale > 0 and finite, growth_factor >= 1,
+ * 0 < backoff_factor <= 1 and growth_interval >= 1. */
+ZERO_API zero_status zero_opt_state_init_dynamic(void* opt_state, float initial_scale, float growth_factor,
+                                                 float backoff_factor, int32_t growth_interval, void* stream);
 
 /* Bytes of scratch a zero_shard_step call with these arguments needs (the
  * workspace fields of args are ignored).  A few hundred bytes in SPECULATIVE

@@ -69,7 +69,9 @@ class GpuResult:
 
 
 def run_gpu(pb: Problem, hp: B.HParams, *, layout=B.ZERO_GRADS_FULL, owner_first=0,
-            owner_count=None, stage=1, steps=None, check_guards=True) -> GpuResult:
+            owner_count=None, stage=1, steps=None, check_guards=True, dynamic=None) -> GpuResult:
+    """dynamic: (initial_scale, growth_factor, backoff_factor, growth_interval)
+    switches dynamic loss scaling on."""
     nd, psi = pb.nd, pb.psi
     oc = nd if owner_count is None else owner_count
     o0 = owner_first
@@ -119,7 +121,10 @@ def run_gpu(pb: Problem, hp: B.HParams, *, layout=B.ZERO_GRADS_FULL, owner_first
         args.workspace = ws.data_ptr()
         args.workspace_bytes = ws_bytes
         stream = torch.cuda.current_stream().cuda_stream
-        B.zero_opt_state_init(opt_state.data_ptr(), stream)
+        if dynamic is None:
+            B.zero_opt_state_init(opt_state.data_ptr(), stream)
+        else:
+            B.zero_opt_state_init_dynamic(opt_state.data_ptr(), *dynamic, stream=stream)
         results = []
         n_steps = len(pb.grads) if steps is None else steps
         for t in range(n_steps):
@@ -162,8 +167,9 @@ class OracleResult:
 
 
 def run_oracle(pb: Problem, hp: oracle.HP, lo=0, hi=None, steps=None, clip_overrides=None,
-               threads=1) -> OracleResult:
-    """The oracle's step over flat range [lo, hi) (the owners of one call)."""
+               threads=1, dynamic=None) -> OracleResult:
+    """The oracle's step over flat range [lo, hi) (the owners of one call).
+    Each info also records the loss scale after its step."""
     hi = pb.psi if hi is None else hi
     master = pb.master[lo:hi].copy()
     m = pb.exp_avg[lo:hi].copy()
@@ -171,6 +177,9 @@ def run_oracle(pb: Problem, hp: oracle.HP, lo=0, hi=None, steps=None, clip_overr
     params = pb.params.copy()
     sub_p = params[lo:hi].copy()
     opt = oracle.Opt()
+    if dynamic is not None:
+        opt = oracle.Opt(loss_scale=dynamic[0], growth_factor=dynamic[1], backoff_factor=dynamic[2],
+                         growth_interval=dynamic[3])
     infos = []
     n_steps = len(pb.grads) if steps is None else steps
     for t in range(n_steps):
@@ -179,6 +188,7 @@ def run_oracle(pb: Problem, hp: oracle.HP, lo=0, hi=None, steps=None, clip_overr
         if hi > lo:
             infos.append(oracle.step(G, master, m, v, sub_p, hp, opt, clip_override=c,
                                      threads=threads))
+            infos[-1]["loss_scale"] = opt.loss_scale
         else:
             infos.append({"overflow": 0})
             opt.t += 1

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
     lib = B.lib()
     for name in declared:
         assert getattr(lib, name) is not None
-    assert B.zero_abi_version() == 2
+    assert B.zero_abi_version() == 3
     # nothing else leaks out of the library (hidden visibility)
     assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
 
@@ -58,7 +58,8 @@ int main(void) {
   S(zero_opt_state) S(zero_step_result) S(zero_hparams) S(zero_step_args)
   O(zero_step_args, master) O(zero_step_args, params) O(zero_step_args, workspace_bytes)
   O(zero_step_args, timing_events) O(zero_hparams, mode) O(zero_opt_state, cur)
-  O(zero_step_result, overflow) O(zero_step_result, status) O(zero_plan_desc, nd) O(zero_plan_info, nd)
+  O(zero_step_result, overflow) O(zero_step_result, status) O(zero_step_result, loss_scale)
+  O(zero_opt_state, loss_scale) O(zero_opt_state, growth_interval) O(zero_plan_desc, nd) O(zero_plan_info, nd)
   return 0;
 }
 """

@@ -236,8 +236,8 @@ def test_checkpoint_resume_equals_uninterrupted():
         g_dev = dev(pb.grads[1])
         opt_state = torch.zeros(B.OPT_STATE_BYTES, dtype=torch.uint8, device="cuda")
         raw = bytearray(B.OPT_STATE_BYTES)
-        saved = first.opt
-        raw[:40] = bytes(saved)
+        saved = bytes(first.opt)          # the checkpointed optimizer state
+        raw[:len(saved)] = saved
         opt_state.copy_(torch.frombuffer(raw, dtype=torch.uint8))
         args = B.step_args(grads=g_dev.data_ptr(), grad_rank_stride=pb.grads[1].shape[1],
                            master=(master.data_ptr(), 0), exp_avg=(m.data_ptr(), 0),
@@ -316,3 +316,25 @@ def test_launch_counter_counts_kernels():
     run_gpu(pb, B.hparams(loss_scale=1024.0, mode=B.ZERO_MODE_STASH, max_grad_norm=1.0))
     # init + prep + 4 statistics launches (one per bucket) + finalize + update
     assert B.zero_launch_count() - before == 8
+
+
+@pytest.mark.parametrize("mode", MODES, ids=lambda m: MODE_NAMES[m])
+@pytest.mark.parametrize("layout", [B.ZERO_GRADS_FULL, B.ZERO_GRADS_PER_OWNER], ids=["full", "per_owner"])
+def test_dynamic_loss_scaling_sequence(mode, layout):
+    """Dynamic loss scale in the device optimizer state: 8 steps with two
+    injected overflows and growth after 2 clean steps; scale, counters and
+    state track the oracle step by step."""
+    S0 = 2.0 ** 12
+    pb = make_problem(70_001, 4, align=256, steps=8, seed=81, S=S0)
+    for t, (r, i) in ((2, (1, 5_000)), (5, (3, 70_000))):
+        pb.grads[t][r, i] = 0x7C00
+    dyn = (S0, 2.0, 0.5, 2)
+    clip = 0.0 if mode == B.ZERO_MODE_SPECULATIVE else 1e-3
+    hp = B.hparams(loss_scale=1.0, weight_decay=0.01, max_grad_norm=clip, mode=mode)
+    g = run_gpu(pb, hp, layout=layout, stage=3 if layout else 1, dynamic=dyn)
+    o = run_oracle(pb, to_oracle_hp(hp), dynamic=dyn,
+                   clip_overrides=None if not clip else [r.clip_coef for r in g.results])
+    compare(g, o, "dynamic scale")
+    assert [r.overflow for r in g.results] == [0, 0, 1, 0, 0, 1, 0, 0]
+    assert [r.loss_scale for r in g.results] == [info["loss_scale"] for info in o.infos]
+    assert [r.loss_scale for r in g.results] == [S0, 2 * S0, S0, S0, 2 * S0, S0, S0, 2 * S0]

@@ -36,7 +36,7 @@ ZERO_GRADS_PER_OWNER = 1
 ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
 ZERO_VOTE_OFFSET = 128               # byte offset of the split step's fp64[2] vote in the workspace
 
-OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (40 bytes used)
+OPT_STATE_BYTES = 64   # device allocation for zero_opt_state (64 bytes)
 RESULT_BYTES = 64      # device allocation for zero_step_result (40 bytes used)
 
 
@@ -75,13 +75,15 @@ class StateReport(C.Structure):
 
 class OptState(C.Structure):
     _fields_ = [("t", C.c_int64), ("beta1_pow", C.c_double), ("beta2_pow", C.c_double),
-                ("skipped", C.c_int64), ("cur", C.c_int32), ("reserved", C.c_int32)]
+                ("skipped", C.c_int64), ("cur", C.c_int32), ("reserved", C.c_int32),
+                ("loss_scale", C.c_float), ("good_steps", C.c_int32), ("growth_factor", C.c_float),
+                ("backoff_factor", C.c_float), ("growth_interval", C.c_int32), ("reserved2", C.c_int32)]
 
 
 class StepResult(C.Structure):
     _fields_ = [("grad_norm", C.c_double), ("t", C.c_int64), ("skipped", C.c_int64),
                 ("clip_coef", C.c_float), ("overflow", C.c_int32), ("status", C.c_int32),
-                ("reserved", C.c_int32)]
+                ("loss_scale", C.c_float)]
 
 
 class HParams(C.Structure):
@@ -116,6 +118,7 @@ SIGNATURES = {
     "zero_plan_destroy": (None, [_P]),
     "zero_state_bytes": (_S, [C.c_int64, C.c_int32, C.c_int32, C.c_int64, C.POINTER(StateReport)]),
     "zero_opt_state_init": (_S, [_P, _P]),
+    "zero_opt_state_init_dynamic": (_S, [_P, C.c_float, C.c_float, C.c_float, C.c_int32, _P]),
     "zero_workspace_bytes": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), C.POINTER(C.c_size_t)]),
     "zero_shard_step": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_static_scratch": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
@@ -144,7 +147,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 2:
+        if L.zero_abi_version() != 3:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -213,6 +216,13 @@ def zero_state_bytes(psi: int, nd: int, stage: int, align_elems: int = 1) -> dic
 
 def zero_opt_state_init(opt_state: int, stream: int = 0) -> None:
     _check(lib().zero_opt_state_init(opt_state, stream), "zero_opt_state_init")
+
+
+def zero_opt_state_init_dynamic(opt_state: int, initial_scale: float, growth_factor: float = 2.0,
+                                backoff_factor: float = 0.5, growth_interval: int = 2000,
+                                stream: int = 0) -> None:
+    _check(lib().zero_opt_state_init_dynamic(opt_state, initial_scale, growth_factor, backoff_factor,
+                                             growth_interval, stream), "zero_opt_state_init_dynamic")
 
 
 def zero_workspace_bytes(plan: int, hp: HParams, args: StepArgs) -> int:

@@ -189,9 +189,27 @@ zero_status zero_opt_state_init(void* opt_state, void* stream)
         return fail(ZERO_ERR_INVALID_ARG, "zero_opt_state_init: null opt_state");
     if (!aligned(opt_state, 8))
         return fail(ZERO_ERR_ALIGNMENT, "zero_opt_state_init: opt_state must be 8-byte aligned");
-    cudaError_t e = zs::launch_opt_init(static_cast<zero_opt_state*>(opt_state),
+    cudaError_t e = zs::launch_opt_init(static_cast<zero_opt_state*>(opt_state), 0.0f, 2.0f, 0.5f, 2000,
                                         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? ZERO_OK : cuda_fail(e, "zero_opt_state_init");
+}
+
+zero_status zero_opt_state_init_dynamic(void* opt_state, float initial_scale, float growth_factor,
+                                        float backoff_factor, int32_t growth_interval, void* stream)
+{
+    zs::clear_error();
+    if (!opt_state)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_opt_state_init_dynamic: null opt_state");
+    if (!aligned(opt_state, 8))
+        return fail(ZERO_ERR_ALIGNMENT, "zero_opt_state_init_dynamic: opt_state must be 8-byte aligned");
+    if (!(initial_scale > 0.0f) || !std::isfinite(initial_scale) || !(growth_factor >= 1.0f) ||
+        !std::isfinite(growth_factor) || !(backoff_factor > 0.0f && backoff_factor <= 1.0f) ||
+        growth_interval < 1)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_opt_state_init_dynamic: need scale > 0, growth >= 1, "
+                    "0 < backoff <= 1, interval >= 1");
+    cudaError_t e = zs::launch_opt_init(static_cast<zero_opt_state*>(opt_state), initial_scale, growth_factor,
+                                        backoff_factor, growth_interval, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : cuda_fail(e, "zero_opt_state_init_dynamic");
 }
 
 zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hparams* hp,
@@ -268,7 +286,8 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
     const bool first_half = phase != PHASE_END;
     const bool second_half = phase != PHASE_BEGIN;
     cudaError_t e;
-    if (first_half && (e = zs::launch_prep(st, ws, h.beta1, h.beta2, str)) != cudaSuccess)
+    const double scale_mult = h.average_over_nd ? (double)p.nd : 1.0;
+    if (first_half && (e = zs::launch_prep(st, ws, h.beta1, h.beta2, u.inv, scale_mult, str)) != cudaSuccess)
         return cuda_fail(e, "prep launch");
 
     if (spec) {
@@ -303,6 +322,8 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
         sa.ws = ws;
         sa.nd = p.nd;
         sa.inv = u.inv;
+        sa.st = st;
+        sa.scale_mult = scale_mult;
         int64_t n_partials = 0;
         for (const auto& b : lp.buckets) {
             for (const auto& l : b) {

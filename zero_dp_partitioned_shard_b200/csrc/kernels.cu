@@ -206,6 +206,29 @@ __device__ __forceinline__ void walk_segments(const SegList& segs, ChunkFn&& chu
     }
 }
 
+// Unscale factor of a step: fp32 1/(S [* Nd]) with S the dynamic loss scale
+// when one is in use (computed exactly as the host computes the static one).
+__device__ __forceinline__ float step_inv(const zero_opt_state* st, float static_inv, double scale_mult)
+{
+    const float S = st->loss_scale;
+    return S > 0.0f ? __double2float_rn(__ddiv_rn(1.0, __dmul_rn((double)S, scale_mult))) : static_inv;
+}
+
+// Dynamic loss scaling after a step (nothing when static): back off on a
+// skipped step, grow after growth_interval consecutive applied steps.
+__device__ __forceinline__ void advance_loss_scale(zero_opt_state* st, bool skipped)
+{
+    if (!(st->loss_scale > 0.0f))
+        return;
+    if (skipped) {
+        st->loss_scale = __fmul_rn(st->loss_scale, st->backoff_factor);
+        st->good_steps = 0;
+    } else if (++st->good_steps >= st->growth_interval) {
+        st->loss_scale = __fmul_rn(st->loss_scale, st->growth_factor);
+        st->good_steps = 0;
+    }
+}
+
 __device__ __forceinline__ AdamK load_consts(const UpdateArgs& a, const WsHeader* ws, bool clip)
 {
     AdamK k;
@@ -226,7 +249,7 @@ __device__ __forceinline__ AdamK load_consts(const UpdateArgs& a, const WsHeader
 // K0: optimizer-state init and per-step prep (one thread)
 // ---------------------------------------------------------------------------
 
-__global__ void zs_opt_init_kernel(zero_opt_state* st)
+__global__ void zs_opt_init_kernel(zero_opt_state* st, float scale, float growth, float backoff, int32_t interval)
 {
     st->t = 0;
     st->beta1_pow = 1.0;
@@ -234,12 +257,20 @@ __global__ void zs_opt_init_kernel(zero_opt_state* st)
     st->skipped = 0;
     st->cur = 0;
     st->reserved = 0;
+    st->loss_scale = scale; // 0: static scaling
+    st->good_steps = 0;
+    st->growth_factor = growth;
+    st->backoff_factor = backoff;
+    st->growth_interval = interval;
+    st->reserved2 = 0;
 }
 
 // Bias corrections of the step about to be applied, from the fp64 running
 // products beta^t: bc = (fp32)(1 - beta^(t+1)).
-__global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2)
+__global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2, float static_inv,
+                               double scale_mult)
 {
+    ws->inv = step_inv(st, static_inv, scale_mult); // the update kernels' unscale factor
     const double b1 = __dmul_rn(st->beta1_pow, (double)beta1);
     const double b2 = __dmul_rn(st->beta2_pow, (double)beta2);
     ws->overflow = 0u;
@@ -264,15 +295,15 @@ __global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float bet
 // finite (only meaningful when the reduced gradient is computed here).
 template <int SRC>
 __device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg, int64_t e, const AdamK& k,
-                                              const float* p_in, const float* m_in, const float* v_in,
-                                              float* p_out, float* m_out, float* v_out)
+                                              float inv, const float* p_in, const float* m_in,
+                                              const float* v_in, float* p_out, float* m_out, float* v_out)
 {
     const int64_t so = sg.s_off + e;
     float g;
     if (SRC == kSrcStash)
         g = a.stash[so];
     else
-        g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
+        g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
     float p = p_in[so], m = m_in[so], v = v_in[so];
     adam_update(__fmul_rn(g, k.clip), p, m, v, k);
     p_out[so] = p;
@@ -295,6 +326,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
     const int cur = kSpec ? ws->cur : 0;
     const int nxt = kSpec ? cur ^ 1 : 0;
     const AdamK k = load_consts(a, ws, !kSpec);
+    const float inv = ws->inv;
     // slot selection by value: indexing the parameter arrays with a runtime
     // index would force a local-memory copy of the whole argument struct
     const float* __restrict__ p_in = cur ? a.master[1] : a.master[0];
@@ -319,7 +351,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
                 rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                    g[q] = __fmul_rn(g[q], a.inv);
+                    g[q] = __fmul_rn(g[q], inv);
             }
             if (kSpec) {
 #pragma unroll
@@ -335,7 +367,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8(p));
         },
         [&](const Seg& sg, int64_t e) {
-            bad |= update_scalar<SRC>(a, sg, e, k, p_in, m_in, v_in, p_out, m_out, v_out);
+            bad |= update_scalar<SRC>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
         });
     if (kSpec)
         flag_nonfinite(bad, &a.ws->overflow);
@@ -593,6 +625,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
     } else {
         // ---- consumers ----
         const AdamK k = load_consts(a, ws, !kSpec);
+        const float inv = ws->inv;
         const int c = threadIdx.x; // 0 .. kPipeConsumers-1
         bool bad = false;
         int it = 0;
@@ -629,7 +662,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                     }
 #pragma unroll
                     for (int q = 0; q < EPT; ++q)
-                        gr[q] = __fmul_rn(gr[q], a.inv);
+                        gr[q] = __fmul_rn(gr[q], inv);
                 }
                 if (kSpec) {
 #pragma unroll
@@ -656,7 +689,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 const Seg& sg = segs.seg[si];
                 const int64_t e = (sg.n >> 3) * 8 + gtid;
                 if (e < sg.n)
-                    bad |= update_scalar<SRC>(a, sg, e, k, p_in, m_in, v_in, p_out, m_out, v_out);
+                    bad |= update_scalar<SRC>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
             }
         }
         if (kSpec)
@@ -684,6 +717,9 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
     // overlap at their boundaries while completion stays ordered (the flag was
     // reset by the prep kernel that heads the chain).
     allow_dependents();
+    // The loss scale comes from the optimizer state: only the previous
+    // step's last kernels wrote it, and they completed before this step began.
+    const float inv = step_inv(a.st, a.inv, a.scale_mult);
     double acc = 0.0;
     bool bad = false;
     walk_segments<VEC>(
@@ -693,7 +729,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
             rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                g[q] = __fmul_rn(g[q], a.inv);
+                g[q] = __fmul_rn(g[q], inv);
                 bad |= !isfinite(g[q]);
                 const double d = (double)g[q];
                 acc = __dadd_rn(acc, __dmul_rn(d, d));
@@ -702,7 +738,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
                 st_f8(a.stash + sg.s_off + e, g);
         },
         [&](const Seg& sg, int64_t e) {
-            const float g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), a.inv);
+            const float g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
             bad |= !isfinite(g);
             const double d = (double)g;
             acc = __dadd_rn(acc, __dmul_rn(d, d));
@@ -779,6 +815,9 @@ __device__ __forceinline__ void decide_step(WsHeader* ws, double sumsq, bool ski
     } else {
         st->skipped += 1;
     }
+    // No reader of this step's scale is left: the statistics launches are
+    // complete and the update reads the prep kernel's snapshot.
+    advance_loss_scale(st, skip);
     if (res) {
         res->grad_norm = skip ? __longlong_as_double(0x7ff8000000000000LL) : norm;
         res->t = st->t;
@@ -786,7 +825,7 @@ __device__ __forceinline__ void decide_step(WsHeader* ws, double sumsq, bool ski
         res->clip_coef = clip;
         res->overflow = skip ? 1 : 0;
         res->status = ZERO_OK;
-        res->reserved = 0;
+        res->loss_scale = st->loss_scale;
     }
 }
 
@@ -868,6 +907,8 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
         } else {
             st->skipped += 1;
         }
+        if (!fault) // the update that read this step's scale has completed
+            advance_loss_scale(st, over);
         if (res) {
             res->grad_norm = __longlong_as_double(0x7ff8000000000000LL);
             res->t = st->t;
@@ -875,7 +916,7 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
             res->clip_coef = 1.0f;
             res->overflow = ws->overflow != 0u ? 1 : 0;
             res->status = fault ? ZERO_ERR_TIMEOUT : ZERO_OK;
-            res->reserved = 0;
+            res->loss_scale = st->loss_scale;
         }
     }
     if (!over)
@@ -1028,17 +1069,18 @@ static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, u
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
 }
 
-cudaError_t launch_opt_init(zero_opt_state* st, cudaStream_t s)
+cudaError_t launch_opt_init(zero_opt_state* st, float scale, float growth, float backoff, int32_t interval,
+                            cudaStream_t s)
 {
-    zs_opt_init_kernel<<<1, 1, 0, s>>>(st);
+    zs_opt_init_kernel<<<1, 1, 0, s>>>(st, scale, growth, backoff, interval);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2,
-                        cudaStream_t s)
+cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2, float static_inv,
+                        double scale_mult, cudaStream_t s)
 {
-    zs_prep_kernel<<<1, 1, 0, s>>>(st, ws, beta1, beta2);
+    zs_prep_kernel<<<1, 1, 0, s>>>(st, ws, beta1, beta2, static_inv, scale_mult);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -65,7 +65,9 @@ struct WsHeader {
     double b1p_next, b2p_next;
     double sumsq, norm;
     int64_t t_next;
-    unsigned char pad1[ZERO_VOTE_OFFSET - 72];
+    float inv;      // unscale factor of this step: fp32 1/(S [* Nd]), S static or dynamic
+    int32_t pad2;
+    unsigned char pad1[ZERO_VOTE_OFFSET - 80];
     double vote[2]; // split step: {sum of squares, non-finite seen}, at ZERO_VOTE_OFFSET
 };
 static_assert(sizeof(WsHeader) <= kHeaderBytes, "workspace header too large");
@@ -99,8 +101,10 @@ struct StatsArgs {
     float* stash; // nullptr unless STASH
     WsHeader* ws;
     double* partials;
+    const zero_opt_state* st; // the dynamic loss scale, when in use
+    double scale_mult;        // Nd when averaging, else 1
     int32_t nd;
-    float inv;
+    float inv;                // static unscale factor
 };
 
 struct GatherEntry {
@@ -116,9 +120,10 @@ struct GatherList {
 };
 
 // ---- launchers (kernels.cu); each returns the launch's cudaError_t ----------
-cudaError_t launch_opt_init(zero_opt_state* st, cudaStream_t s);
-cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2,
-                        cudaStream_t s);
+cudaError_t launch_opt_init(zero_opt_state* st, float scale, float growth, float backoff, int32_t interval,
+                            cudaStream_t s);
+cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2, float static_inv,
+                        double scale_mult, cudaStream_t s);
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs,
                           cudaStream_t s);
 // blocks (= fp64 partials written) of one statistics launch over segs
