@@ -380,6 +380,46 @@ void oracle_gather_params(const uint16_t* const* shards, const oracle_plan_t* p,
     }
 }
 
+/* On-demand gather of a tensor range (stage 3: a layer's parameters are
+ * gathered when the forward or backward pass reaches it, then released --
+ * [Dissect] "ZeRO-3" and the figure under "Forward/Backward Under ZeRO-3").
+ * Tensors first .. first + count - 1 of the flat layout (sizes as in
+ * oracle_tensor_segments) are assembled from the owners' fp16 shards: the
+ * element at flat index f comes from shards[f / L][f % L].  compact = 0: into
+ * `out` at the flat index (a Psi-element buffer), where a NULL shard means
+ * that owner's part is already in place and is left untouched; compact = 1:
+ * tensors back to back from out[0], every needed shard required.  Returns
+ * the number of elements copied, -1 on bad arguments (sizes not adding up to
+ * Psi, range outside the list, or a shard missing in compact mode). */
+int64_t oracle_gather_tensors(const oracle_plan_t* p, const int64_t* sizes, int32_t n_tensors,
+                              int32_t first, int32_t count, const uint16_t* const* shards,
+                              uint16_t* out, int32_t compact)
+{
+    int64_t total = 0;
+    for (int32_t t = 0; t < n_tensors; ++t)
+        total += sizes[t];
+    if (total != p->psi || first < 0 || count < 0 || first + count > n_tensors)
+        return -1;
+    int64_t flat = 0, written = 0;
+    for (int32_t t = 0; t < first; ++t)
+        flat += sizes[t];
+    for (int32_t t = first; t < first + count; ++t) {
+        for (int64_t j = 0; j < sizes[t]; ++j) {
+            const int64_t f = flat + j;
+            const int64_t owner = f / p->shard_len;
+            if (!shards[owner]) {
+                if (compact)
+                    return -1;
+                continue;
+            }
+            out[compact ? written : f] = shards[owner][f - owner * p->shard_len];
+            ++written;
+        }
+        flat += sizes[t];
+    }
+    return written;
+}
+
 /* ------------------------------------------------------------------------ */
 /* The shard step                                                            */
 /* ------------------------------------------------------------------------ */

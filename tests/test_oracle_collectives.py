@@ -73,3 +73,49 @@ def test_gather_params_rebuilds_the_flat_buffer():
         mask = np.ones(psi, bool)
         mask[s:s + n] = False
         assert np.array_equal(full2[mask], ref[mask])
+
+
+def test_gather_tensors_equals_slices_of_the_full_gather():
+    """Gathering a tensor range (compact or in place) gives exactly the slices
+    of the fully gathered buffer; every tensor range together is everything."""
+    rs = np.random.default_rng(19)
+    for trial in range(25):
+        sizes = [int(x) for x in rs.integers(0, 400, size=int(rs.integers(1, 15)))]
+        psi = sum(sizes)
+        if psi == 0:
+            continue
+        nd = int(rs.integers(1, 7))
+        p = oracle.plan(psi, nd, int(rs.choice([1, 8, 32])))
+        ref = synth.fp16_bits(synth.normal_f32(psi, seed=trial, std=1.0))
+        shards = []
+        for r in range(nd):
+            st, n = p.shard(r)
+            sh = np.full(p.shard_len, 0x7E00, np.uint16)
+            sh[:n] = ref[st:st + n]
+            shards.append(sh)
+        offs = np.concatenate([[0], np.cumsum(sizes)])
+        first = int(rs.integers(0, len(sizes)))
+        count = int(rs.integers(0, len(sizes) - first + 1))
+        lo, hi = int(offs[first]), int(offs[first + count])
+        compact = np.zeros(max(hi - lo, 1), np.uint16)
+        assert oracle.gather_tensors(shards, p, sizes, first, count, compact, True) == hi - lo
+        assert np.array_equal(compact[:hi - lo], ref[lo:hi])
+        full = np.full(psi, 0x1234, np.uint16)
+        oracle.gather_tensors(shards, p, sizes, first, count, full, False)
+        assert np.array_equal(full[lo:hi], ref[lo:hi])
+        assert (full[:lo] == 0x1234).all() and (full[hi:] == 0x1234).all()
+        # in place, a missing shard's part is left as it is
+        skip = int(rs.integers(0, nd))
+        part = np.full(psi, 0x1234, np.uint16)
+        n_copied = oracle.gather_tensors([None if r == skip else shards[r] for r in range(nd)], p,
+                                         sizes, first, count, part, False)
+        s0, n0 = p.shard(skip)
+        owned = np.zeros(psi, bool)
+        owned[s0:s0 + n0] = True
+        inside = np.zeros(psi, bool)
+        inside[lo:hi] = True
+        assert np.array_equal(part[inside & ~owned], ref[inside & ~owned])
+        assert (part[~inside | owned] == 0x1234).all()
+        assert n_copied == int((inside & ~owned).sum())
+    with pytest.raises(ValueError):
+        oracle.gather_tensors([None] * p.nd, p, sizes, 0, len(sizes), np.zeros(psi, np.uint16), True)
