@@ -366,6 +366,23 @@ ZERO_API zero_status zero_shard_step_static_scratch(const zero_plan_t* plan, con
 ZERO_API zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard_ptrs,
                                void* params_full, void* stream);
 
+/* On-demand gather of a tensor range, for stage 3: a layer's parameters are
+ * gathered when the forward or backward pass reaches them and released after
+ * use ("ZeRO memory optimization", trishampatil.com, "ZeRO-3" and the figure
+ * under "Forward/Backward Under ZeRO-3").  Tensors first_tensor ..
+ * first_tensor + n_tensors - 1 of the plan's tensor list (the plan must have
+ * one) are assembled from the owners' fp16 shards (shard_ptrs: host array of
+ * nd device pointers, [L] each): the element at flat index f comes from
+ * shard f / L at f % L.  compact = 0: into `out` (device fp16, Psi elements)
+ * at the flat index; a NULL shard is then skipped (its part is already in
+ * place).  compact = 1: tensors back to back from out[0] (device fp16, the
+ * range's element count); every needed shard must be given.  *elements
+ * (host, may be NULL) receives the number of elements copied -- the gather's
+ * communication volume when the shards live on other processes. */
+ZERO_API zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                         const void* const* shard_ptrs, void* out, int32_t compact,
+                                         int64_t* elements, void* stream);
+
 /* params[(owner_first + j) * L + i] = fp16(master[j * L + i]) for the owners
  * owner_first .. owner_first + owner_count - 1: establishes the fp16 copy
  * of a freshly initialised fp32 master (device pointers). */

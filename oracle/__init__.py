@@ -89,6 +89,7 @@ def lib():
             "oracle_reduce_scatter": (None, [_P, _I64, C.POINTER(PlanT), _P]),
             "oracle_all_gather_f32": (None, [_P, C.POINTER(PlanT), _P]),
             "oracle_gather_params": (None, [_P, C.POINTER(PlanT), _P]),
+            "oracle_gather_tensors": (_I64, [C.POINTER(PlanT), _P, _I32, _I32, _I32, _P, _P, _I32]),
             "oracle_bias_corrections": (None, [C.POINTER(HParams), C.POINTER(OptState),
                                                C.POINTER(C.c_double), C.POINTER(C.c_double),
                                                C.POINTER(C.c_float), C.POINTER(C.c_float)]),
@@ -232,6 +233,29 @@ def gather_params(shards, p: Plan, full: np.ndarray) -> np.ndarray:
     pc = p._c()
     lib().oracle_gather_params(ptrs, C.byref(pc), _ptr(full))
     return full
+
+
+def gather_tensors(shards, p: Plan, sizes, first: int, count: int, out: np.ndarray,
+                   compact: bool) -> int:
+    """Assembles tensors first..first+count-1 from the owners' fp16 shards
+    (list of nd uint16 arrays or None) into ``out``; returns elements written."""
+    sizes = np.ascontiguousarray(sizes, dtype=np.int64)
+    keep = []
+    ptrs = (C.c_void_p * p.nd)()
+    for r, sh in enumerate(shards):
+        if sh is None:
+            ptrs[r] = None
+        else:
+            sh = np.ascontiguousarray(sh, dtype=np.uint16)
+            keep.append(sh)
+            ptrs[r] = sh.ctypes.data
+    assert out.dtype == np.uint16 and out.flags["C_CONTIGUOUS"]
+    pc = p._c()
+    n = lib().oracle_gather_tensors(C.byref(pc), _ptr(sizes), len(sizes), first, count, ptrs,
+                                    _ptr(out), int(compact))
+    if n < 0:
+        raise ValueError("gather_tensors: bad range, sizes or missing shard")
+    return n
 
 
 # --------------------------------------------------------------------------

@@ -251,3 +251,21 @@ def test_wait_budget_hook_round_trips():
     assert B.zero_set_wait_budget(-1) == 12345
     assert B.zero_set_wait_budget(0) == -1
     assert B.zero_set_wait_budget(0) == 1 << 31
+
+
+def test_gather_tensors_validation():
+    no_list = B.zero_plan(100, 2, align_elems=8)
+    with_list = B.zero_plan(100, 2, align_elems=8, tensor_sizes=[30, 30, 40])
+    try:
+        for plan, first, count in ((no_list, 0, 1), (with_list, 2, 2), (with_list, -1, 1)):
+            before = B.zero_launch_count()
+            with pytest.raises(B.ZeroError) as e:
+                B.zero_gather_tensors(plan, first, count, [FAKE, FAKE], FAKE, True)
+            assert e.value.status == B.ZERO_ERR_INVALID_ARG
+            assert B.zero_launch_count() == before
+        with pytest.raises(B.ZeroError) as e:    # compact gather with a missing owner shard
+            B.zero_gather_tensors(with_list, 0, 3, [FAKE, 0], FAKE, True)
+        assert e.value.status == B.ZERO_ERR_INVALID_ARG
+    finally:
+        B.zero_plan_destroy(no_list)
+        B.zero_plan_destroy(with_list)

@@ -125,6 +125,7 @@ SIGNATURES = {
     "zero_shard_step_begin": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_end": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
+    "zero_gather_tensors": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, _P]),
     "zero_abi_version": (C.c_int32, []),
     "zero_strerror": (C.c_char_p, [_S]),
@@ -256,6 +257,16 @@ def zero_gather_params(plan: int, shard_ptrs, params_full: int, stream: int = 0)
     arr = (C.c_void_p * len(shard_ptrs))(*[p if p else None for p in shard_ptrs])
     _check(lib().zero_gather_params(plan, C.cast(arr, C.c_void_p), params_full, stream),
            "zero_gather_params")
+
+
+def zero_gather_tensors(plan: int, first_tensor: int, n_tensors: int, shard_ptrs, out: int,
+                        compact: bool, stream: int = 0) -> int:
+    """Gathers a tensor range from the owners' shards; returns the elements copied."""
+    arr = (C.c_void_p * len(shard_ptrs))(*[p if p else None for p in shard_ptrs])
+    n = C.c_int64()
+    _check(lib().zero_gather_tensors(plan, first_tensor, n_tensors, C.cast(arr, C.c_void_p), out,
+                                     int(compact), C.byref(n), stream), "zero_gather_tensors")
+    return n.value
 
 
 def zero_cast_params(plan: int, master: int, params: int, owner_first: int, owner_count: int,

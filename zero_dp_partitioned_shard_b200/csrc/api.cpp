@@ -374,6 +374,29 @@ zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hparams* hp,
     return run_step(plan, hp, args, stream, PHASE_END);
 }
 
+// Launches copies of shard pieces, at most kMaxSegs per launch.
+static zero_status launch_pieces(std::vector<zs::GatherEntry>& entries, uint16_t* dst, cudaStream_t str,
+                                 const char* what)
+{
+    for (size_t i = 0; i < entries.size(); i += zs::kMaxSegs) {
+        zs::GatherList g;
+        std::memset(&g, 0, sizeof g);
+        for (size_t k = i; k < entries.size() && g.count < zs::kMaxSegs; ++k)
+            g.e[g.count++] = entries[k];
+        cudaError_t e = zs::launch_gather(dst, g, str);
+        if (e != cudaSuccess)
+            return cuda_fail(e, what);
+    }
+    return ZERO_OK;
+}
+
+static zs::GatherEntry piece(const void* src, int64_t src_off, const void* dst, int64_t dst_off, int64_t n)
+{
+    const uint16_t* s = static_cast<const uint16_t*>(src) + src_off;
+    const uint16_t* d = static_cast<const uint16_t*>(dst) + dst_off;
+    return zs::GatherEntry{s, dst_off, n, (aligned(s, 16) && aligned(d, 16)) ? 1 : 0};
+}
+
 zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard_ptrs,
                                void* params_full, void* stream)
 {
@@ -384,7 +407,6 @@ zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard
     if (!aligned(params_full, 2))
         return fail(ZERO_ERR_ALIGNMENT, "zero_gather_params: params_full must be 2-byte aligned");
     std::vector<zs::GatherEntry> entries;
-    bool vec = (p.shard_len % 8 == 0) && aligned(params_full, 16);
     for (int32_t r = 0; r < p.nd; ++r) {
         if (!shard_ptrs[r])
             continue;
@@ -393,22 +415,55 @@ zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard
         const int64_t start = (int64_t)r * p.shard_len;
         int64_t n = p.psi - start;
         n = n < 0 ? 0 : (n > p.shard_len ? p.shard_len : n);
-        if (n == 0)
+        if (n > 0)
+            entries.push_back(piece(shard_ptrs[r], 0, params_full, start, n));
+    }
+    return launch_pieces(entries, static_cast<uint16_t*>(params_full), static_cast<cudaStream_t>(stream),
+                         "gather launch");
+}
+
+zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                const void* const* shard_ptrs, void* out, int32_t compact,
+                                int64_t* elements, void* stream)
+{
+    zs::clear_error();
+    if (!plan || !shard_ptrs || !out)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: null argument");
+    const zero_plan_s& p = *plan;
+    const int32_t nt = (int32_t)p.tensor_offset.size() - 1;
+    if (nt < 1)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: the plan was built without a tensor list");
+    if (first_tensor < 0 || n_tensors < 0 || first_tensor > nt - n_tensors)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: tensors [%d, %d + %d) outside [0, %d)",
+                    first_tensor, first_tensor, n_tensors, nt);
+    if (compact != 0 && compact != 1)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: compact must be 0 or 1");
+    if (!aligned(out, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "zero_gather_tensors: out must be 2-byte aligned");
+    const int64_t base = p.tensor_offset[(size_t)first_tensor];
+    std::vector<zs::GatherEntry> entries;
+    int64_t n_elems = 0;
+    for (const zero_segment& sg : p.segments) {
+        if (sg.tensor < first_tensor || sg.tensor >= first_tensor + n_tensors)
             continue;
-        vec = vec && aligned(shard_ptrs[r], 16);
-        entries.push_back({static_cast<const uint16_t*>(shard_ptrs[r]), start, n});
+        const void* sh = shard_ptrs[sg.owner];
+        const int64_t flat = p.tensor_offset[(size_t)sg.tensor] + sg.offset_in_tensor;
+        if (!sh) {
+            if (compact)
+                return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: tensor %lld needs owner %lld's shard",
+                            (long long)sg.tensor, (long long)sg.owner);
+            continue; // in place: this owner's part is already there
+        }
+        if (!aligned(sh, 2))
+            return fail(ZERO_ERR_ALIGNMENT, "zero_gather_tensors: shard %lld must be 2-byte aligned",
+                        (long long)sg.owner);
+        entries.push_back(piece(sh, sg.offset_in_shard, out, compact ? flat - base : flat, sg.length));
+        n_elems += sg.length;
     }
-    cudaStream_t str = static_cast<cudaStream_t>(stream);
-    for (size_t i = 0; i < entries.size(); i += zs::kMaxSegs) {
-        zs::GatherList g;
-        std::memset(&g, 0, sizeof g);
-        for (size_t k = i; k < entries.size() && g.count < zs::kMaxSegs; ++k)
-            g.e[g.count++] = entries[k];
-        cudaError_t e = zs::launch_gather(vec, static_cast<uint16_t*>(params_full), g, str);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "gather launch");
-    }
-    return ZERO_OK;
+    if (elements)
+        *elements = n_elems;
+    return launch_pieces(entries, static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream),
+                         "gather launch");
 }
 
 zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,

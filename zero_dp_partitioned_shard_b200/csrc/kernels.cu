@@ -935,37 +935,35 @@ zs_cast_kernel(const float* master, uint16_t* params, const __grid_constant__ Se
 // K4: gather-assembly of fp16 parameter shards into the full buffer
 // ---------------------------------------------------------------------------
 
-template <bool VEC>
 __global__ void __launch_bounds__(kThreads)
 zs_gather_kernel(uint16_t* dst, const __grid_constant__ GatherList g)
 {
-    // the shards' 8-element chunks as one index space (see walk_segments)
+    // the pieces' units -- 8-element vectors for aligned pieces, single
+    // elements otherwise -- as one grid-stride index space (see walk_segments)
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    const int shift = VEC ? 3 : 0;
     int64_t total = 0;
     for (int k = 0; k < g.count; ++k)
-        total += g.e[k].n >> shift;
+        total += g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n;
     int k = 0;
     int64_t base = 0;
     for (int64_t u = tid; u < total; u += nthr) {
-        while (u >= base + (g.e[k].n >> shift)) {
-            base += g.e[k].n >> shift;
+        while (u >= base + (g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n)) {
+            base += g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n;
             ++k;
         }
         const GatherEntry& ge = g.e[k];
-        if (VEC)
-            __stcs(reinterpret_cast<uint4*>(dst + ge.dst_off) + (u - base), ld_stream(ge.src + ((u - base) << 3)));
+        const int64_t i = u - base;
+        if (ge.vec)
+            __stcs(reinterpret_cast<uint4*>(dst + ge.dst_off) + i, ld_stream(ge.src + (i << 3)));
         else
-            dst[ge.dst_off + (u - base)] = ge.src[u - base];
+            dst[ge.dst_off + i] = ge.src[i];
     }
-    if (VEC) {
-        for (int j = 0; j < g.count; ++j) {
-            const GatherEntry& ge = g.e[j];
-            const int64_t e = ((ge.n >> 3) << 3) + tid;
-            if (e < ge.n)
-                dst[ge.dst_off + e] = ge.src[e];
-        }
+    for (int j = 0; j < g.count; ++j) { // tails of the vector pieces
+        const GatherEntry& ge = g.e[j];
+        const int64_t e = ((ge.n >> 3) << 3) + tid;
+        if (ge.vec && e < ge.n)
+            dst[ge.dst_off + e] = ge.src[e];
     }
 }
 
@@ -1284,20 +1282,16 @@ cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const S
     return cudaGetLastError();
 }
 
-cudaError_t launch_gather(bool vec, uint16_t* dst, const GatherList& g, cudaStream_t s)
+cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s)
 {
     int64_t w = 0;
     for (int i = 0; i < g.count; ++i)
-        w += vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
+        w += g.e[i].vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
     int blocks = 0;
-    cudaError_t e = vec ? grid_for(zs_gather_kernel<true>, w, 0, &blocks)
-                        : grid_for(zs_gather_kernel<false>, w, 0, &blocks);
+    cudaError_t e = grid_for(zs_gather_kernel, w, 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    if (vec)
-        zs_gather_kernel<true><<<blocks, kThreads, 0, s>>>(dst, g);
-    else
-        zs_gather_kernel<false><<<blocks, kThreads, 0, s>>>(dst, g);
+    zs_gather_kernel<<<blocks, kThreads, 0, s>>>(dst, g);
     count_launches(1);
     return cudaGetLastError();
 }

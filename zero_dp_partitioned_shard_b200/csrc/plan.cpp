@@ -119,6 +119,7 @@ zero_status zero_plan(const zero_plan_desc* d, zero_plan_t** out)
         const int64_t L = p->shard_len;
         for (int32_t t = 0; t < d->n_tensors; ++t) {
             const int64_t size = d->tensor_sizes[t];
+            p->tensor_offset.push_back(base);
             for (int64_t done = 0; done < size;) {
                 const int64_t flat = base + done;
                 const int64_t owner = flat / L;
@@ -129,6 +130,7 @@ zero_status zero_plan(const zero_plan_desc* d, zero_plan_t** out)
             }
             base += size;
         }
+        p->tensor_offset.push_back(base);
     }
     *out = p;
     return ZERO_OK;

@@ -20,6 +20,7 @@ struct zero_plan_s {
     int32_t nd = 1;
     int32_t stage = 0;
     std::vector<zero_segment> segments; // tensor -> owner pieces (optional)
+    std::vector<int64_t> tensor_offset;  // flat offset of each tensor, plus psi at the end
 };
 
 namespace zs {
@@ -111,6 +112,7 @@ struct GatherEntry {
     const uint16_t* src;
     int64_t dst_off;
     int64_t n;
+    int64_t vec; // 1: src and dst + dst_off 16-byte aligned, copied in 8-element vectors
 };
 
 struct GatherList {
@@ -139,6 +141,6 @@ cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bo
                           zero_opt_state* st, zero_step_result* res, cudaStream_t s);
 cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
                         cudaStream_t s);
-cudaError_t launch_gather(bool vec, uint16_t* dst, const GatherList& g, cudaStream_t s);
+cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s);
 
 } // namespace zs
