@@ -46,7 +46,7 @@ class HParams(C.Structure):
         ("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float),
         ("eps", C.c_float), ("weight_decay", C.c_float),
         ("loss_scale", C.c_float), ("max_grad_norm", C.c_float),
-        ("average_over_nd", C.c_int32),
+        ("average_over_nd", C.c_int32), ("storage", C.c_int32),
     ]
 
 
@@ -79,6 +79,8 @@ def lib():
             "oracle_half_to_float": (C.c_float, [C.c_uint16]),
             "oracle_float_to_half": (C.c_uint16, [C.c_float]),
             "oracle_half_to_float_array": (None, [_P, _P, _I64]),
+            "oracle_bf16_to_float_array": (None, [_P, _P, _I64]),
+            "oracle_float_to_bf16_array": (None, [_P, _P, _I64]),
             "oracle_float_to_half_array": (None, [_P, _P, _I64]),
             "oracle_plan": (C.c_int, [_I64, _I32, _I64, _I64, C.POINTER(PlanT)]),
             "oracle_shard": (None, [C.POINTER(PlanT), _I32, C.POINTER(_I64), C.POINTER(_I64)]),
@@ -123,6 +125,20 @@ def half_to_float(h: np.ndarray) -> np.ndarray:
     h = np.ascontiguousarray(h, dtype=np.uint16)
     out = np.empty(h.shape, dtype=np.float32)
     lib().oracle_half_to_float_array(_ptr(h), _ptr(out), h.size)
+    return out
+
+
+def bf16_to_float(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float32)
+    lib().oracle_bf16_to_float_array(_ptr(h), _ptr(out), h.size)
+    return out
+
+
+def float_to_bf16(f: np.ndarray) -> np.ndarray:
+    f = np.ascontiguousarray(f, dtype=np.float32)
+    out = np.empty(f.shape, dtype=np.uint16)
+    lib().oracle_float_to_bf16_array(_ptr(f), _ptr(out), f.size)
     return out
 
 
@@ -272,10 +288,12 @@ class HP:
     loss_scale: float = 1.0
     max_grad_norm: float = 0.0
     average_over_nd: bool = False
+    storage: int = 0          # 16-bit format of gradients and parameters: 0 fp16, 1 bf16
 
     def _c(self) -> HParams:
         return HParams(self.lr, self.beta1, self.beta2, self.eps, self.weight_decay,
-                       self.loss_scale, self.max_grad_norm, int(self.average_over_nd))
+                       self.loss_scale, self.max_grad_norm, int(self.average_over_nd),
+                       int(self.storage))
 
 
 @dataclasses.dataclass

@@ -24,7 +24,8 @@
  *
  * Precision.  The pages fix the storage types ([Dissect] "The Real Problem",
  * 16-Psi equation; [Note] Concepts, mixed precision): fp16 parameters and
- * gradients, fp32 master copy, momentum and variance.  The update is therefore
+ * gradients, fp32 master copy, momentum and variance.  bfloat16 (the same
+ * 2 bytes) is supported as an alternative 16-bit format.  The update is therefore
  * done in fp32 with every operation separately rounded (built with
  * -ffp-contract=off, no fast-math, SSE arithmetic so no excess precision).
  *
@@ -129,6 +130,39 @@ uint16_t oracle_float_to_half(float f)
     uint32_t q = full >> drop;
     q = round_nearest_even(q, full & ((1u << drop) - 1u), drop);
     return (uint16_t)(sign | q); /* q == 0x400 is the smallest normal */
+}
+
+/* bfloat16: the upper 16 bits of a binary32 (same exponent range, 8-bit
+ * significand).  Widening is exact. */
+float oracle_bf16_to_float(uint16_t h)
+{
+    uint32_t bits = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return f;
+}
+
+/* binary32 -> bfloat16, round to nearest even on the 16 dropped bits
+ * (subnormals kept, overflow to infinity, NaN kept quiet). */
+uint16_t oracle_float_to_bf16(float f)
+{
+    uint32_t x;
+    memcpy(&x, &f, sizeof x);
+    if ((x & 0x7F800000u) == 0x7F800000u && (x & 0x7FFFFFu))
+        return (uint16_t)((x >> 16) | 0x0040u);
+    return (uint16_t)round_nearest_even(x >> 16, x & 0xFFFFu, 16);
+}
+
+void oracle_bf16_to_float_array(const uint16_t* h, float* f, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        f[i] = oracle_bf16_to_float(h[i]);
+}
+
+void oracle_float_to_bf16_array(const float* f, uint16_t* h, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        h[i] = oracle_float_to_bf16(f[i]);
 }
 
 void oracle_half_to_float_array(const uint16_t* h, float* f, int64_t n)
@@ -314,20 +348,32 @@ int oracle_state_bytes(int64_t psi, int32_t nd, int32_t stage, int64_t align, or
 /* Collectives, written out as their definitions                            */
 /* ------------------------------------------------------------------------ */
 
-/* Contribution of rank r at flat index i: rank r's fp16 buffer starts
- * rank_stride elements after rank r-1's. */
-static float contribution(const uint16_t* G, int64_t rank_stride, int32_t r, int64_t i)
+/* Contribution of rank r at flat index i: rank r's 16-bit buffer starts
+ * rank_stride elements after rank r-1's (storage 0: fp16, 1: bf16). */
+static float contribution(const uint16_t* G, int64_t rank_stride, int32_t r, int64_t i, int32_t storage)
 {
-    return oracle_half_to_float(G[(int64_t)r * rank_stride + i]);
+    const uint16_t h = G[(int64_t)r * rank_stride + i];
+    return storage ? oracle_bf16_to_float(h) : oracle_half_to_float(h);
 }
 
 /* Sum over ranks 0..Nd-1 at index i, left to right in fp32. */
+static float rank_sum_of(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t i, int32_t storage)
+{
+    float s = contribution(G, rank_stride, 0, i, storage);
+    for (int32_t r = 1; r < nd; ++r)
+        s = s + contribution(G, rank_stride, r, i, storage);
+    return s;
+}
+
 static float rank_sum(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t i)
 {
-    float s = contribution(G, rank_stride, 0, i);
-    for (int32_t r = 1; r < nd; ++r)
-        s = s + contribution(G, rank_stride, r, i);
-    return s;
+    return rank_sum_of(G, rank_stride, nd, i, 0);
+}
+
+/* The cast of an updated master value into the parameter format. */
+static uint16_t to_storage(float p, int32_t storage)
+{
+    return storage ? oracle_float_to_bf16(p) : oracle_float_to_half(p);
 }
 
 /* All-reduce: every process ends with the full sum ([Note] Key results: DP's
@@ -429,6 +475,7 @@ typedef struct {
     float loss_scale;    /* S: contributions carry the loss scaled by S */
     float max_grad_norm; /* <= 0: no clipping */
     int32_t average_over_nd;
+    int32_t storage;     /* 16-bit format of gradients and parameters: 0 fp16, 1 bf16 */
 } oracle_hparams;
 
 typedef struct {
@@ -577,10 +624,10 @@ void oracle_update_elements(const uint16_t* G, int64_t rank_stride, int32_t nd, 
     (void)threads;
 #pragma omp parallel for num_threads(threads > 0 ? threads : 1) if (threads > 1) schedule(static)
     for (int64_t i = 0; i < n; ++i) {
-        float g = rank_sum(G, rank_stride, nd, i) * inv;
+        float g = rank_sum_of(G, rank_stride, nd, i, hp->storage) * inv;
         float g_hat = g * k.clip;
         adam_element(g_hat, &master[i], &exp_avg[i], &exp_avg_sq[i], &k);
-        params[i] = oracle_float_to_half(master[i]);
+        params[i] = to_storage(master[i], hp->storage);
     }
 }
 
@@ -609,7 +656,7 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
     /* 1. reduce-scatter sum (every owner's slice) and unscale */
 #pragma omp parallel for num_threads(threads > 0 ? threads : 1) if (threads > 1) schedule(static)
     for (int64_t i = 0; i < psi; ++i)
-        g[i] = rank_sum(G, rank_stride, nd, i) * inv;
+        g[i] = rank_sum_of(G, rank_stride, nd, i, hp->storage) * inv;
 
     /* 2. overflow: one non-finite element anywhere skips the whole step */
     int32_t overflow = 0;
@@ -655,7 +702,7 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
     for (int64_t i = 0; i < psi; ++i) {
         float g_hat = g[i] * k.clip;
         adam_element(g_hat, &master[i], &exp_avg[i], &exp_avg_sq[i], &k);
-        params[i] = oracle_float_to_half(master[i]);
+        params[i] = to_storage(master[i], hp->storage);
     }
 
     st->t += 1;
@@ -681,7 +728,7 @@ double oracle_grad_sumsq(const uint16_t* G, int64_t rank_stride, int32_t nd, int
     const float inv = unscale_factor(hp, nd);
     comp_sum a = {acc, 0.0};
     for (int64_t i = 0; i < n; ++i) {
-        float g = rank_sum(G, rank_stride, nd, i) * inv;
+        float g = rank_sum_of(G, rank_stride, nd, i, hp->storage) * inv;
         if (!isfinite(g))
             *nonfinite = 1;
         comp_add(&a, (double)g * (double)g);

@@ -314,3 +314,23 @@ def test_static_scale_leaves_the_scale_state_alone():
     oracle.step(G, synth.normal_f32(100, seed=1, std=0.02), np.zeros(100, F32), np.zeros(100, F32),
                 np.zeros(100, np.uint16), oracle.HP(loss_scale=8.0), opt)
     assert (opt.loss_scale, opt.good_steps, opt.t) == (0.0, 0, 1)
+
+
+def test_bf16_storage_step_matches_its_definition():
+    """With bf16 gradients and parameters the step is the same arithmetic with
+    bf16 widening of the contributions and a bf16 cast of the master."""
+    nd, n, S = 4, 2000, 1.0
+    G32 = (synth.normal_f32(nd * n, seed=91, std=1e-3) * np.float32(S)).reshape(nd, n)
+    G = oracle.float_to_bf16(G32)
+    hp = oracle.HP(loss_scale=S, weight_decay=0.01, storage=1)
+    master = synth.normal_f32(n, seed=92, std=0.02)
+    m, v, P = np.zeros(n, F32), np.zeros(n, F32), np.zeros(n, np.uint16)
+    m0 = master.copy()
+    oracle.step(G, master, m, v, P, hp, oracle.Opt())
+    # the reduced gradient is the rank-order fp32 sum of the widened bf16 values
+    g = oracle.bf16_to_float(G[0])
+    for r in range(1, nd):
+        g = (g + oracle.bf16_to_float(G[r])).astype(F32)
+    assert (m == (F32(1.0 - F32(0.9)) * g).astype(F32)).all()
+    assert np.array_equal(P, oracle.float_to_bf16(master))
+    assert not np.array_equal(master, m0)

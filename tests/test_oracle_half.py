@@ -74,3 +74,40 @@ def test_specials():
     want = vals.astype(np.float16).view(np.uint16)
     assert np.array_equal(got, want)
     assert got[1] == 0x8000 and got[4] == 0x7BFF and got[5] == 0x7C00 and got[8] == 0
+
+
+# --- bfloat16: pinned against torch's bfloat16 casts (a library routine) ---
+
+def _torch_bf16_bits(x32):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x32, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_bf16_to_float_all_65536_patterns():
+    import torch
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = oracle.bf16_to_float(h)
+    want = torch.from_numpy(h.view(np.int16)).view(torch.bfloat16).float().numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(got[~nan].view(np.uint32), want[~nan].view(np.uint32))
+    assert np.isnan(got[nan]).all()
+
+
+def _check_f32_to_bf16(bits):
+    x = bits.astype(np.uint32).view(np.float32)
+    got = oracle.float_to_bf16(x)
+    want = _torch_bf16_bits(x)
+    nan = np.isnan(x)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert (((got[nan] & 0x7F80) == 0x7F80) & ((got[nan] & 0x7F) != 0)).all()
+
+
+def test_float_to_bf16_rounding_boundaries_every_prefix():
+    hi = np.arange(1 << 16, dtype=np.uint64) << 16
+    for lo in (0x0000, 0x0001, 0x7FFF, 0x8000, 0x8001, 0xFFFF, 0x4000, 0xC000):
+        _check_f32_to_bf16(hi | lo)
+
+
+def test_float_to_bf16_random_patterns():
+    rs = np.random.default_rng(17)
+    _check_f32_to_bf16(rs.integers(0, 1 << 32, size=1 << 22, dtype=np.uint64))
