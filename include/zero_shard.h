@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 3
+#define ZERO_SHARD_ABI_VERSION 4
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -110,6 +110,13 @@ typedef int32_t zero_status;
  *     (0 means L). */
 #define ZERO_GRADS_FULL 0
 #define ZERO_GRADS_PER_OWNER 1
+
+/* 16-bit format of the gradient contributions and of the parameters.  The
+ * pages' mixed precision uses fp16; bfloat16 (the same 2 bytes, the upper half
+ * of a binary32) is the alternative.  Widening is exact for both, narrowing
+ * rounds to nearest even; the step's arithmetic is otherwise identical. */
+#define ZERO_STORAGE_FP16 0
+#define ZERO_STORAGE_BF16 1
 
 /* ---- plan ------------------------------------------------------------------ */
 /* Partition of Psi parameters over Nd owners ("ZeRO memory optimization",
@@ -254,7 +261,7 @@ typedef struct zero_step_args {
     int32_t grad_layout;
     int32_t owner_first;
     int32_t owner_count;
-    int32_t reserved;
+    int32_t storage;        /* ZERO_STORAGE_FP16 or ZERO_STORAGE_BF16 (grads and params) */
     float* master[2];
     float* exp_avg[2];
     float* exp_avg_sq[2];
@@ -383,11 +390,12 @@ ZERO_API zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_
                                          const void* const* shard_ptrs, void* out, int32_t compact,
                                          int64_t* elements, void* stream);
 
-/* params[(owner_first + j) * L + i] = fp16(master[j * L + i]) for the owners
- * owner_first .. owner_first + owner_count - 1: establishes the fp16 copy
- * of a freshly initialised fp32 master (device pointers). */
+/* params[(owner_first + j) * L + i] = cast(master[j * L + i]) for the owners
+ * owner_first .. owner_first + owner_count - 1, in the 16-bit format
+ * `storage` (ZERO_STORAGE_*): establishes the 16-bit copy of a freshly
+ * initialised fp32 master (device pointers). */
 ZERO_API zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,
-                             int32_t owner_first, int32_t owner_count, void* stream);
+                             int32_t owner_first, int32_t owner_count, int32_t storage, void* stream);
 
 /* ---- diagnostics ---------------------------------------------------------------- */
 ZERO_API int32_t zero_abi_version(void);

@@ -37,14 +37,21 @@ class Problem:
     exp_avg: np.ndarray
     exp_avg_sq: np.ndarray
     params: np.ndarray     # uint16 [psi]
+    storage: int = 0       # 16-bit format of grads and params (B.ZERO_STORAGE_*)
+
+
+# a quiet NaN in each 16-bit format, for pads the kernels must not read
+NAN16 = {B.ZERO_STORAGE_FP16: np.uint16(0x7E00), B.ZERO_STORAGE_BF16: np.uint16(0x7FC0)}
+INF16 = {B.ZERO_STORAGE_FP16: np.uint16(0x7C00), B.ZERO_STORAGE_BF16: np.uint16(0x7F80)}
 
 
 def make_problem(psi, nd, align=256, bucket=0, steps=1, seed=0, S=1024.0, std=1e-3,
-                 random_state=False, pad_fill=np.nan):
+                 random_state=False, pad_fill=np.nan, storage=B.ZERO_STORAGE_FP16):
     from zero_dp_partitioned_shard_b200 import synth
     pl = oracle.plan(psi, nd, align, bucket)
-    grads = [synth.grads_f16(nd, psi, seed=seed * 100 + t, std=std, scale=S, stride=pl.psi_pad,
-                             pad_fill=pad_fill) for t in range(steps)]
+    draw = synth.grads_bf16 if storage == B.ZERO_STORAGE_BF16 else synth.grads_f16
+    grads = [draw(nd, psi, seed=seed * 100 + t, std=std, scale=S, stride=pl.psi_pad,
+                  pad_fill=pad_fill) for t in range(steps)]
     master = synth.normal_f32(psi, seed=seed * 100 + 91, std=0.02)
     if random_state:
         m = synth.normal_f32(psi, seed=seed * 100 + 92, std=1e-4)
@@ -52,8 +59,8 @@ def make_problem(psi, nd, align=256, bucket=0, steps=1, seed=0, S=1024.0, std=1e
     else:
         m = np.zeros(psi, np.float32)
         v = np.zeros(psi, np.float32)
-    params = synth.fp16_bits(master)
-    return Problem(psi, nd, align, bucket, grads, master, m, v, params)
+    params = synth.bf16_bits(master) if storage == B.ZERO_STORAGE_BF16 else synth.fp16_bits(master)
+    return Problem(psi, nd, align, bucket, grads, master, m, v, params, storage)
 
 
 @dataclasses.dataclass
@@ -99,7 +106,7 @@ def run_gpu(pb: Problem, hp: B.HParams, *, layout=B.ZERO_GRADS_FULL, owner_first
         def grads_buf(G):
             if layout == B.ZERO_GRADS_FULL:
                 return dev(G), G.shape[1]
-            blk = np.full((oc, nd, L), np.float16(np.nan).view(np.uint16), dtype=np.uint16)
+            blk = np.full((oc, nd, L), NAN16[pb.storage], dtype=np.uint16)
             for j in range(oc):
                 s = (o0 + j) * L
                 n = max(0, min(L, psi - s))
@@ -115,7 +122,7 @@ def run_gpu(pb: Problem, hp: B.HParams, *, layout=B.ZERO_GRADS_FULL, owner_first
                            master=(ptr(master[0]), ptr(master[1])), exp_avg=(ptr(m[0]), ptr(m[1])),
                            exp_avg_sq=(ptr(v[0]), ptr(v[1])), params=params.data_ptr(),
                            grad_stash=ptr(stash), opt_state=opt_state.data_ptr(),
-                           result=result.data_ptr())
+                           result=result.data_ptr(), storage=pb.storage)
         ws_bytes = B.zero_workspace_bytes(plan, hp, args)
         ws = torch.empty(ws_bytes + 4096, dtype=torch.uint8, device="cuda")
         args.workspace = ws.data_ptr()
@@ -196,7 +203,8 @@ def run_oracle(pb: Problem, hp: oracle.HP, lo=0, hi=None, steps=None, clip_overr
     return OracleResult(master, m, v, params, infos, opt)
 
 
-def to_oracle_hp(hp: B.HParams) -> oracle.HP:
+def to_oracle_hp(hp: B.HParams, storage: int = B.ZERO_STORAGE_FP16) -> oracle.HP:
     return oracle.HP(lr=hp.lr, beta1=hp.beta1, beta2=hp.beta2, eps=hp.eps,
                      weight_decay=hp.weight_decay, loss_scale=hp.loss_scale,
-                     max_grad_norm=hp.max_grad_norm, average_over_nd=bool(hp.average_over_nd))
+                     max_grad_norm=hp.max_grad_norm, average_over_nd=bool(hp.average_over_nd),
+                     storage=storage)

@@ -45,6 +45,18 @@ def assert_f16_close(got_bits, want_bits, max_ulp, what=""):
     assert worst <= max_ulp, f"{what}: {worst} fp16 ulp > {max_ulp} (at {int(np.argmax(d))})"
 
 
+def assert_bf16_close(got_bits, want_bits, max_ulp, what=""):
+    got = np.asarray(got_bits, np.uint16)
+    want = np.asarray(want_bits, np.uint16)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    nan_g = ((got & 0x7F80) == 0x7F80) & ((got & 0x7F) != 0)
+    nan_w = ((want & 0x7F80) == 0x7F80) & ((want & 0x7F) != 0)
+    assert np.array_equal(nan_g, nan_w), f"{what}: NaN positions differ"
+    d = ulp16(got[~nan_g], want[~nan_w])   # sign-magnitude order holds for both formats
+    worst = int(d.max()) if d.size else 0
+    assert worst <= max_ulp, f"{what}: {worst} bf16 ulp > {max_ulp} (at {int(np.argmax(d))})"
+
+
 def read_golden(path):
     """Parse a golden fixture: '#' comments, then whitespace-separated rows."""
     rows = []

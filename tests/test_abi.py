@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
     lib = B.lib()
     for name in declared:
         assert getattr(lib, name) is not None
-    assert B.zero_abi_version() == 3
+    assert B.zero_abi_version() == 4
     # nothing else leaks out of the library (hidden visibility)
     assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
 
@@ -174,7 +174,7 @@ def _args(**kw):
     ("stash_missing", B.ZERO_ERR_INVALID_ARG), ("misaligned_master", B.ZERO_ERR_ALIGNMENT),
     ("misaligned_params", B.ZERO_ERR_ALIGNMENT), ("small_ws", B.ZERO_ERR_WORKSPACE),
     ("null_ws", B.ZERO_ERR_WORKSPACE), ("misaligned_ws", B.ZERO_ERR_ALIGNMENT),
-    ("reserved", B.ZERO_ERR_INVALID_ARG),
+    ("reserved", B.ZERO_ERR_INVALID_ARG), ("bad_storage", B.ZERO_ERR_INVALID_ARG),
 ])
 def test_step_validation_rejects_before_launch(case, status):
     plan = B.zero_plan(1000, 4, stage=1, align_elems=8)
@@ -213,8 +213,10 @@ def test_step_validation_rejects_before_launch(case, status):
     elif case == "misaligned_ws":
         args = _args(workspace=FAKE + 16)
     elif case == "reserved":
+        hp.reserved = 1
+    elif case == "bad_storage":
         args = _args()
-        args.reserved = 1
+        args.storage = 2
     before = B.zero_launch_count()
     try:
         with pytest.raises(B.ZeroError) as e:

@@ -33,6 +33,9 @@ ZERO_MODE_STASH = 2
 ZERO_GRADS_FULL = 0
 ZERO_GRADS_PER_OWNER = 1
 
+ZERO_STORAGE_FP16 = 0
+ZERO_STORAGE_BF16 = 1
+
 ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
 ZERO_VOTE_OFFSET = 128               # byte offset of the split step's fp64[2] vote in the workspace
 
@@ -96,7 +99,7 @@ class HParams(C.Structure):
 class StepArgs(C.Structure):
     _fields_ = [("grads", C.c_void_p), ("grad_rank_stride", C.c_int64),
                 ("grad_layout", C.c_int32), ("owner_first", C.c_int32),
-                ("owner_count", C.c_int32), ("reserved", C.c_int32),
+                ("owner_count", C.c_int32), ("storage", C.c_int32),
                 ("master", C.c_void_p * 2), ("exp_avg", C.c_void_p * 2),
                 ("exp_avg_sq", C.c_void_p * 2), ("params", C.c_void_p),
                 ("grad_stash", C.c_void_p), ("opt_state", C.c_void_p), ("result", C.c_void_p),
@@ -126,7 +129,7 @@ SIGNATURES = {
     "zero_shard_step_end": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
     "zero_gather_tensors": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
-    "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, _P]),
+    "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, C.c_int32, _P]),
     "zero_abi_version": (C.c_int32, []),
     "zero_strerror": (C.c_char_p, [_S]),
     "zero_last_error": (C.c_char_p, []),
@@ -148,7 +151,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 3:
+        if L.zero_abi_version() != 4:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -270,8 +273,8 @@ def zero_gather_tensors(plan: int, first_tensor: int, n_tensors: int, shard_ptrs
 
 
 def zero_cast_params(plan: int, master: int, params: int, owner_first: int, owner_count: int,
-                     stream: int = 0) -> None:
-    _check(lib().zero_cast_params(plan, master, params, owner_first, owner_count, stream),
+                     stream: int = 0, storage: int = ZERO_STORAGE_FP16) -> None:
+    _check(lib().zero_cast_params(plan, master, params, owner_first, owner_count, storage, stream),
            "zero_cast_params")
 
 
@@ -310,7 +313,7 @@ def hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0, loss_sc
 def step_args(*, grads: int, grad_rank_stride: int, master, exp_avg, exp_avg_sq, params: int,
               opt_state: int, workspace: int = 0, workspace_bytes: int = 0, result: int = 0,
               grad_layout: int = ZERO_GRADS_FULL, owner_first: int = 0, owner_count: int = 1,
-              grad_stash: int = 0, timing_events=(0, 0)) -> StepArgs:
+              grad_stash: int = 0, timing_events=(0, 0), storage: int = ZERO_STORAGE_FP16) -> StepArgs:
     """master/exp_avg/exp_avg_sq: (slot0, slot1) device addresses (slot1 may be 0)."""
     a = StepArgs()
     a.grads = grads
@@ -318,7 +321,7 @@ def step_args(*, grads: int, grad_rank_stride: int, master, exp_avg, exp_avg_sq,
     a.grad_layout = grad_layout
     a.owner_first = owner_first
     a.owner_count = owner_count
-    a.reserved = 0
+    a.storage = storage
     for k in range(2):
         a.master[k] = master[k] or None
         a.exp_avg[k] = exp_avg[k] or None

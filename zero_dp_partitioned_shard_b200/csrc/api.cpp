@@ -75,8 +75,10 @@ zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_st
         return fail(ZERO_ERR_INVALID_ARG, "zero_shard_step: null plan, hparams or args");
     if (hp->mode < ZERO_MODE_SPECULATIVE || hp->mode > ZERO_MODE_STASH)
         return fail(ZERO_ERR_INVALID_ARG, "unknown mode %d", hp->mode);
-    if (hp->reserved != 0 || a->reserved != 0)
+    if (hp->reserved != 0)
         return fail(ZERO_ERR_INVALID_ARG, "reserved fields must be 0");
+    if (a->storage != ZERO_STORAGE_FP16 && a->storage != ZERO_STORAGE_BF16)
+        return fail(ZERO_ERR_INVALID_ARG, "unknown 16-bit storage format %d", a->storage);
     if (!(hp->loss_scale > 0.0f) || !std::isfinite(hp->loss_scale))
         return fail(ZERO_ERR_INVALID_ARG, "loss_scale must be finite and > 0");
     if (!std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay) || !std::isfinite(hp->eps) ||
@@ -268,6 +270,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
     u.ws = ws;
     u.result = res;
     u.wait_budget = zs::wait_budget_cycles();
+    u.bf16 = a.storage == ZERO_STORAGE_BF16 ? 1 : 0;
     u.nd = p.nd;
     double scale = (double)h.loss_scale;
     if (h.average_over_nd)
@@ -324,6 +327,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
         sa.inv = u.inv;
         sa.st = st;
         sa.scale_mult = scale_mult;
+        sa.bf16 = u.bf16;
         int64_t n_partials = 0;
         for (const auto& b : lp.buckets) {
             for (const auto& l : b) {
@@ -467,11 +471,13 @@ zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, i
 }
 
 zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,
-                             int32_t owner_first, int32_t owner_count, void* stream)
+                             int32_t owner_first, int32_t owner_count, int32_t storage, void* stream)
 {
     zs::clear_error();
     if (!plan || !master || !params)
         return fail(ZERO_ERR_INVALID_ARG, "zero_cast_params: null argument");
+    if (storage != ZERO_STORAGE_FP16 && storage != ZERO_STORAGE_BF16)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_cast_params: unknown 16-bit storage format %d", storage);
     const zero_plan_s& p = *plan;
     if (owner_first < 0 || owner_count < 1 || owner_first > p.nd - owner_count)
         return fail(ZERO_ERR_INVALID_ARG, "zero_cast_params: owner range outside the plan");
@@ -485,7 +491,7 @@ zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void*
     const bool vec = (p.shard_len % 8 == 0) && aligned(master, 16) && aligned(params, 16) &&
                      segs_vec_ok(lists);
     for (const auto& l : lists) {
-        cudaError_t e = zs::launch_cast(vec, master, static_cast<uint16_t*>(params), l,
+        cudaError_t e = zs::launch_cast(vec, storage == ZERO_STORAGE_BF16, master, static_cast<uint16_t*>(params), l,
                                         static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess)
             return cuda_fail(e, "cast launch");

@@ -26,6 +26,7 @@
 // intrinsic (no contraction into FMA), division and square root are the
 // IEEE-rounded __fdiv_rn / __fsqrt_rn, and the fp16 cast is round-to-nearest-
 // even with subnormals kept.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <map>
@@ -60,25 +61,46 @@ __device__ __forceinline__ void adam_update(float g, float& p, float& m, float& 
     v = v_new;
 }
 
+// 16-bit storage formats: BF = false is IEEE binary16, BF = true is
+// bfloat16 (the upper half of a binary32, so widening is a shift).  Narrowing
+// rounds to nearest even in both.
+template <bool BF>
 __device__ __forceinline__ void unpack_h8(const uint4& x, float f[8])
 {
-    const __half2* h = reinterpret_cast<const __half2*>(&x);
+    if (BF) {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float2 t = __half22float2(h[q]);
-        f[2 * q] = t.x;
-        f[2 * q + 1] = t.y;
+        for (int q = 0; q < 4; ++q) {
+            f[2 * q] = __uint_as_float(w[q] << 16);
+            f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+        }
+    } else {
+        const __half2* h = reinterpret_cast<const __half2*>(&x);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 t = __half22float2(h[q]);
+            f[2 * q] = t.x;
+            f[2 * q + 1] = t.y;
+        }
     }
 }
 
+template <bool BF>
+__device__ __forceinline__ uint32_t pack_h2(float a, float b)
+{
+    if (BF) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <bool BF>
 __device__ __forceinline__ uint4 pack_h8(const float f[8])
 {
-    uint4 x;
-    __half2* h = reinterpret_cast<__half2*>(&x);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        h[q] = __floats2half2_rn(f[2 * q], f[2 * q + 1]);
-    return x;
+    return make_uint4(pack_h2<BF>(f[0], f[1]), pack_h2<BF>(f[2], f[3]), pack_h2<BF>(f[4], f[5]),
+                      pack_h2<BF>(f[6], f[7]));
 }
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p)
@@ -100,12 +122,21 @@ __device__ __forceinline__ void st_f8(float* p, const float f[8])
     __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(f[4], f[5], f[6], f[7]));
 }
 
-__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+template <bool BF>
+__device__ __forceinline__ float h2f(uint16_t h)
+{
+    return BF ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
+}
 
-__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+template <bool BF>
+__device__ __forceinline__ uint16_t f2h(float f)
+{
+    return BF ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
+}
 
 // Rank-order sum of the Nd contributions of 8 consecutive parameters: the
 // loads of each group of 8 ranks are issued together, then added in order.
+template <bool BF>
 __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, int nd, float s[8])
 {
     {
@@ -114,12 +145,12 @@ __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, in
         for (int u = 0; u < 8; ++u)
             if (u < nd)
                 x[u] = ld_stream(g + u * rstride);
-        unpack_h8(x[0], s);
+        unpack_h8<BF>(x[0], s);
 #pragma unroll
         for (int u = 1; u < 8; ++u) {
             if (u < nd) {
                 float f[8];
-                unpack_h8(x[u], f);
+                unpack_h8<BF>(x[u], f);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     s[q] = __fadd_rn(s[q], f[q]);
@@ -136,7 +167,7 @@ __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, in
         for (int u = 0; u < 8; ++u) {
             if (r + u < nd) {
                 float f[8];
-                unpack_h8(x[u], f);
+                unpack_h8<BF>(x[u], f);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     s[q] = __fadd_rn(s[q], f[q]);
@@ -145,11 +176,12 @@ __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, in
     }
 }
 
+template <bool BF>
 __device__ __forceinline__ float rank_sum1(const uint16_t* g, int64_t rstride, int nd)
 {
-    float s = h2f(g[0]);
+    float s = h2f<BF>(g[0]);
     for (int r = 1; r < nd; ++r)
-        s = __fadd_rn(s, h2f(g[(int64_t)r * rstride]));
+        s = __fadd_rn(s, h2f<BF>(g[(int64_t)r * rstride]));
     return s;
 }
 
@@ -293,7 +325,7 @@ __global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float bet
 
 // One element, scalar loads and stores; returns true if its gradient is not
 // finite (only meaningful when the reduced gradient is computed here).
-template <int SRC>
+template <int SRC, bool BF>
 __device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg, int64_t e, const AdamK& k,
                                               float inv, const float* p_in, const float* m_in,
                                               const float* v_in, float* p_out, float* m_out, float* v_out)
@@ -303,17 +335,17 @@ __device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg
     if (SRC == kSrcStash)
         g = a.stash[so];
     else
-        g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
+        g = __fmul_rn(rank_sum1<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
     float p = p_in[so], m = m_in[so], v = v_in[so];
     adam_update(__fmul_rn(g, k.clip), p, m, v, k);
     p_out[so] = p;
     m_out[so] = m;
     v_out[so] = v;
-    a.params[sg.p_off + e] = f2h(p);
+    a.params[sg.p_off + e] = f2h<BF>(p);
     return !isfinite(g);
 }
 
-template <int SRC, bool VEC>
+template <int SRC, bool VEC, bool BF>
 __global__ void __launch_bounds__(kThreads, 2)
 zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
 {
@@ -348,7 +380,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             if (SRC == kSrcStash) {
                 ld_f8(a.stash + so, g);
             } else {
-                rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+                rank_sum8<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     g[q] = __fmul_rn(g[q], inv);
@@ -364,10 +396,10 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             st_f8(p_out + so, p);
             st_f8(m_out + so, m);
             st_f8(v_out + so, v);
-            __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8(p));
+            __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8<BF>(p));
         },
         [&](const Seg& sg, int64_t e) {
-            bad |= update_scalar<SRC>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
+            bad |= update_scalar<SRC, BF>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
         });
     if (kSpec)
         flag_nonfinite(bad, &a.ws->overflow);
@@ -468,21 +500,25 @@ __device__ __forceinline__ void lds_f(const float* p, float f[N])
     }
 }
 
-template <int N>
+template <int N, bool BF>
 __device__ __forceinline__ void lds_h(const uint16_t* p, float f[N])
 {
     if (N == 8) {
-        unpack_h8(*reinterpret_cast<const uint4*>(p), f);
+        unpack_h8<BF>(*reinterpret_cast<const uint4*>(p), f);
     } else if (N == 4) {
         const uint2 x = *reinterpret_cast<const uint2*>(p);
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&x.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&x.y));
-        f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+        const uint32_t w[2] = {x.x, x.y};
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            f[2 * q] = h2f<BF>((uint16_t)(w[q] & 0xFFFFu));
+            f[2 * q + 1] = h2f<BF>((uint16_t)(w[q] >> 16));
+        }
     } else if (N == 2) {
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(p));
-        f[0] = a.x; f[1] = a.y;
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        f[0] = h2f<BF>((uint16_t)(w & 0xFFFFu));
+        f[1] = h2f<BF>((uint16_t)(w >> 16));
     } else {
-        f[0] = h2f(p[0]);
+        f[0] = h2f<BF>(p[0]);
     }
 }
 
@@ -499,22 +535,17 @@ __device__ __forceinline__ void stg_f(float* p, const float f[N])
         __stcs(p, f[0]);
 }
 
-template <int N>
+template <int N, bool BF>
 __device__ __forceinline__ void stg_h(uint16_t* p, const float f[N])
 {
     if (N == 8) {
-        __stcs(reinterpret_cast<uint4*>(p), pack_h8(f));
+        __stcs(reinterpret_cast<uint4*>(p), pack_h8<BF>(f));
     } else if (N == 4) {
-        __half2 h0 = __floats2half2_rn(f[0], f[1]), h1 = __floats2half2_rn(f[2], f[3]);
-        uint2 x;
-        x.x = *reinterpret_cast<uint32_t*>(&h0);
-        x.y = *reinterpret_cast<uint32_t*>(&h1);
-        __stcs(reinterpret_cast<uint2*>(p), x);
+        __stcs(reinterpret_cast<uint2*>(p), make_uint2(pack_h2<BF>(f[0], f[1]), pack_h2<BF>(f[2], f[3])));
     } else if (N == 2) {
-        __half2 h0 = __floats2half2_rn(f[0], f[1]);
-        __stcs(reinterpret_cast<unsigned int*>(p), *reinterpret_cast<unsigned int*>(&h0));
+        __stcs(reinterpret_cast<unsigned int*>(p), pack_h2<BF>(f[0], f[1]));
     } else {
-        p[0] = f2h(f[0]);
+        p[0] = f2h<BF>(f[0]);
     }
 }
 
@@ -527,7 +558,7 @@ __device__ __forceinline__ int tile_segment(const int64_t* first_tile, int count
     return s;
 }
 
-template <int SRC, int EPT>
+template <int SRC, int EPT, bool BF>
 __global__ void __launch_bounds__(kPipeThreads, 2)
 zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages)
 {
@@ -652,10 +683,10 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                     lds_f<EPT>(reinterpret_cast<const float*>(buf + T * 12) + i0, gr);
                 } else {
                     const uint16_t* gs = reinterpret_cast<const uint16_t*>(buf + T * 12) + i0;
-                    lds_h<EPT>(gs, gr);
+                    lds_h<EPT, BF>(gs, gr);
                     for (int r = 1; r < a.nd; ++r) {
                         float f[EPT];
-                        lds_h<EPT>(gs + r * T, f);
+                        lds_h<EPT, BF>(gs + r * T, f);
 #pragma unroll
                         for (int q = 0; q < EPT; ++q)
                             gr[q] = __fadd_rn(gr[q], f[q]);
@@ -676,7 +707,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 stg_f<EPT>(p_out + so, p);
                 stg_f<EPT>(m_out + so, m);
                 stg_f<EPT>(v_out + so, v);
-                stg_h<EPT>(a.params + sg.p_off + e0 + i0, p);
+                stg_h<EPT, BF>(a.params + sg.p_off + e0 + i0, p);
             }
             __syncwarp();
             if (lane == 0)
@@ -689,7 +720,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 const Seg& sg = segs.seg[si];
                 const int64_t e = (sg.n >> 3) * 8 + gtid;
                 if (e < sg.n)
-                    bad |= update_scalar<SRC>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
+                    bad |= update_scalar<SRC, BF>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
             }
         }
         if (kSpec)
@@ -707,7 +738,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
 //     optionally the fp32 reduced gradient (stash)
 // ---------------------------------------------------------------------------
 
-template <bool VEC, bool STASH>
+template <bool VEC, bool STASH, bool BF>
 __global__ void __launch_bounds__(kThreads, 2)
 zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
 {
@@ -726,7 +757,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
         segs,
         [&](const Seg& sg, int64_t e) {
             float g[8];
-            rank_sum8(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+            rank_sum8<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 g[q] = __fmul_rn(g[q], inv);
@@ -738,7 +769,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
                 st_f8(a.stash + sg.s_off + e, g);
         },
         [&](const Seg& sg, int64_t e) {
-            const float g = __fmul_rn(rank_sum1(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
+            const float g = __fmul_rn(rank_sum1<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
             bad |= !isfinite(g);
             const double d = (double)g;
             acc = __dadd_rn(acc, __dmul_rn(d, d));
@@ -875,7 +906,7 @@ __global__ void zs_vote_apply_kernel(WsHeader* ws, int speculative, float max_no
 //     fp16 parameters from the unchanged live master; also zero_cast_params
 // ---------------------------------------------------------------------------
 
-template <bool VEC>
+template <bool VEC, bool BF>
 __device__ __forceinline__ void cast_segments(const float* master, uint16_t* params, const SegList& segs)
 {
     walk_segments<VEC>(
@@ -883,12 +914,12 @@ __device__ __forceinline__ void cast_segments(const float* master, uint16_t* par
         [&](const Seg& sg, int64_t e) {
             float p[8];
             ld_f8(master + sg.s_off + e, p);
-            __stcs(reinterpret_cast<uint4*>(params + sg.p_off + e), pack_h8(p));
+            __stcs(reinterpret_cast<uint4*>(params + sg.p_off + e), pack_h8<BF>(p));
         },
-        [&](const Seg& sg, int64_t e) { params[sg.p_off + e] = f2h(master[sg.s_off + e]); });
+        [&](const Seg& sg, int64_t e) { params[sg.p_off + e] = f2h<BF>(master[sg.s_off + e]); });
 }
 
-template <bool VEC>
+template <bool VEC, bool BF>
 __global__ void __launch_bounds__(kThreads)
 zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int bookkeeping,
                  zero_opt_state* st, zero_step_result* res)
@@ -921,14 +952,14 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
     }
     if (!over)
         return;
-    cast_segments<VEC>(cur ? a.master[1] : a.master[0], a.params, segs);
+    cast_segments<VEC, BF>(cur ? a.master[1] : a.master[0], a.params, segs);
 }
 
-template <bool VEC>
+template <bool VEC, bool BF>
 __global__ void __launch_bounds__(kThreads)
 zs_cast_kernel(const float* master, uint16_t* params, const __grid_constant__ SegList segs)
 {
-    cast_segments<VEC>(master, params, segs);
+    cast_segments<VEC, BF>(master, params, segs);
 }
 
 // ---------------------------------------------------------------------------
@@ -1083,16 +1114,24 @@ cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, flo
     return cudaGetLastError();
 }
 
-template <int SRC, bool VEC>
+template <int SRC, bool VEC, bool BF>
 static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, cudaStream_t s)
 {
     int blocks = 0;
-    cudaError_t e = grid_for(zs_update_kernel<SRC, VEC>, seg_work(segs, VEC), 0, &blocks);
+    cudaError_t e = grid_for(zs_update_kernel<SRC, VEC, BF>, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = launch_overlapped(zs_update_kernel<SRC, VEC>, blocks, kThreads, 0, s, a, segs);
+    e = launch_overlapped(zs_update_kernel<SRC, VEC, BF>, blocks, kThreads, 0, s, a, segs);
     count_launches(1);
     return e;
+}
+
+template <int SRC>
+static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+{
+    if (a.bf16)
+        return vec ? launch_update_t<SRC, true, true>(a, segs, s) : launch_update_t<SRC, false, true>(a, segs, s);
+    return vec ? launch_update_t<SRC, true, false>(a, segs, s) : launch_update_t<SRC, false, false>(a, segs, s);
 }
 
 // Shape of the pipelined update for a given source: elements per consumer
@@ -1129,10 +1168,10 @@ static bool pipe_shape(int src, int nd, PipeShape* ps)
 
 static std::map<std::pair<const void*, int>, int> g_smem_set; // (kernel, device) -> bytes allowed
 
-template <int SRC, int EPT>
+template <int SRC, int EPT, bool BF>
 static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
 {
-    auto kernel = zs_update_pipe_kernel<SRC, EPT>;
+    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF>;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || (e = device_sms(&sms)) != cudaSuccess)
@@ -1160,15 +1199,21 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
     return e;
 }
 
+template <int SRC, bool BF>
+static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+{
+    switch (ps.ept) {
+    case 8: return launch_pipe_t<SRC, 8, BF>(a, segs, ps, s);
+    case 4: return launch_pipe_t<SRC, 4, BF>(a, segs, ps, s);
+    case 2: return launch_pipe_t<SRC, 2, BF>(a, segs, ps, s);
+    default: return launch_pipe_t<SRC, 1, BF>(a, segs, ps, s);
+    }
+}
+
 template <int SRC>
 static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
 {
-    switch (ps.ept) {
-    case 8: return launch_pipe_t<SRC, 8>(a, segs, ps, s);
-    case 4: return launch_pipe_t<SRC, 4>(a, segs, ps, s);
-    case 2: return launch_pipe_t<SRC, 2>(a, segs, ps, s);
-    default: return launch_pipe_t<SRC, 1>(a, segs, ps, s);
-    }
+    return a.bf16 ? launch_pipe_f<SRC, true>(a, segs, ps, s) : launch_pipe_f<SRC, false>(a, segs, ps, s);
 }
 
 // The bulk-copy pipeline pays off where a parameter carries few bytes (the
@@ -1189,15 +1234,9 @@ cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList&
         }
     }
     switch (src) {
-    case kSrcGradsSpeculative:
-        return vec ? launch_update_t<kSrcGradsSpeculative, true>(a, segs, s)
-                   : launch_update_t<kSrcGradsSpeculative, false>(a, segs, s);
-    case kSrcGradsInPlace:
-        return vec ? launch_update_t<kSrcGradsInPlace, true>(a, segs, s)
-                   : launch_update_t<kSrcGradsInPlace, false>(a, segs, s);
-    default:
-        return vec ? launch_update_t<kSrcStash, true>(a, segs, s)
-                   : launch_update_t<kSrcStash, false>(a, segs, s);
+    case kSrcGradsSpeculative: return launch_update_regs<kSrcGradsSpeculative>(vec, a, segs, s);
+    case kSrcGradsInPlace: return launch_update_regs<kSrcGradsInPlace>(vec, a, segs, s);
+    default: return launch_update_regs<kSrcStash>(vec, a, segs, s);
     }
 }
 
@@ -1209,21 +1248,27 @@ int stats_blocks(bool vec, const SegList& segs)
     return (int)(want < 1 ? 1 : (want > kStatsMaxBlocks ? kStatsMaxBlocks : want));
 }
 
-template <bool VEC, bool STASH>
+template <bool VEC, bool STASH, bool BF>
 static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, cudaStream_t s)
 {
-    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH>, stats_blocks(VEC, segs), kThreads, 0, s,
-                                            a, segs);
+    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH, BF>, stats_blocks(VEC, segs), kThreads,
+                                            0, s, a, segs);
     count_launches(1);
     return e;
 }
 
-cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
+template <bool BF>
+static cudaError_t launch_stats_f(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
 {
     const bool stash = a.stash != nullptr;
     if (vec)
-        return stash ? launch_stats_t<true, true>(a, segs, s) : launch_stats_t<true, false>(a, segs, s);
-    return stash ? launch_stats_t<false, true>(a, segs, s) : launch_stats_t<false, false>(a, segs, s);
+        return stash ? launch_stats_t<true, true, BF>(a, segs, s) : launch_stats_t<true, false, BF>(a, segs, s);
+    return stash ? launch_stats_t<false, true, BF>(a, segs, s) : launch_stats_t<false, false, BF>(a, segs, s);
+}
+
+cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
+{
+    return a.bf16 ? launch_stats_f<true>(vec, a, segs, s) : launch_stats_f<false>(vec, a, segs, s);
 }
 
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, float max_norm,
@@ -1251,35 +1296,47 @@ cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, ze
     return cudaGetLastError();
 }
 
-cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
-                          zero_opt_state* st, zero_step_result* res, cudaStream_t s)
+template <bool VEC, bool BF>
+static cudaError_t launch_commit_t(const UpdateArgs& a, const SegList& segs, bool bookkeeping, zero_opt_state* st,
+                                   zero_step_result* res, cudaStream_t s)
 {
     int blocks = 0;
-    cudaError_t e = vec ? grid_for(zs_commit_kernel<true>, seg_work(segs, true), 0, &blocks)
-                        : grid_for(zs_commit_kernel<false>, seg_work(segs, false), 0, &blocks);
+    cudaError_t e = grid_for(zs_commit_kernel<VEC, BF>, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = vec ? launch_overlapped(zs_commit_kernel<true>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res)
-            : launch_overlapped(zs_commit_kernel<false>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st,
-                                res);
+    e = launch_overlapped(zs_commit_kernel<VEC, BF>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res);
     count_launches(1);
     return e;
 }
 
-cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
-                        cudaStream_t s)
+cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
+                          zero_opt_state* st, zero_step_result* res, cudaStream_t s)
+{
+    if (a.bf16)
+        return vec ? launch_commit_t<true, true>(a, segs, bookkeeping, st, res, s)
+                   : launch_commit_t<false, true>(a, segs, bookkeeping, st, res, s);
+    return vec ? launch_commit_t<true, false>(a, segs, bookkeeping, st, res, s)
+               : launch_commit_t<false, false>(a, segs, bookkeeping, st, res, s);
+}
+
+template <bool VEC, bool BF>
+static cudaError_t launch_cast_t(const float* master, uint16_t* params, const SegList& segs, cudaStream_t s)
 {
     int blocks = 0;
-    cudaError_t e = vec ? grid_for(zs_cast_kernel<true>, seg_work(segs, true), 0, &blocks)
-                        : grid_for(zs_cast_kernel<false>, seg_work(segs, false), 0, &blocks);
+    cudaError_t e = grid_for(zs_cast_kernel<VEC, BF>, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    if (vec)
-        zs_cast_kernel<true><<<blocks, kThreads, 0, s>>>(master, params, segs);
-    else
-        zs_cast_kernel<false><<<blocks, kThreads, 0, s>>>(master, params, segs);
+    zs_cast_kernel<VEC, BF><<<blocks, kThreads, 0, s>>>(master, params, segs);
     count_launches(1);
     return cudaGetLastError();
+}
+
+cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
+                        cudaStream_t s)
+{
+    if (bf16)
+        return vec ? launch_cast_t<true, true>(master, params, segs, s) : launch_cast_t<false, true>(master, params, segs, s);
+    return vec ? launch_cast_t<true, false>(master, params, segs, s) : launch_cast_t<false, false>(master, params, segs, s);
 }
 
 cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s)

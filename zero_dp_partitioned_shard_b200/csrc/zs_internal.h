@@ -95,6 +95,7 @@ struct UpdateArgs {
     float one_minus_beta1, one_minus_beta2;
     zero_step_result* result; // receives status = ZERO_ERR_TIMEOUT on a pipeline fault (may be null)
     long long wait_budget;    // cycles per bounded pipeline wait
+    int32_t bf16;             // 16-bit storage of gradients and parameters: 0 fp16, 1 bf16
 };
 
 struct StatsArgs {
@@ -106,6 +107,7 @@ struct StatsArgs {
     double scale_mult;        // Nd when averaging, else 1
     int32_t nd;
     float inv;                // static unscale factor
+    int32_t bf16;             // 16-bit storage of the contributions: 0 fp16, 1 bf16
 };
 
 struct GatherEntry {
@@ -139,7 +141,7 @@ cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, ze
                               zero_step_result* res, cudaStream_t s);
 cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
                           zero_opt_state* st, zero_step_result* res, cudaStream_t s);
-cudaError_t launch_cast(bool vec, const float* master, uint16_t* params, const SegList& segs,
+cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
                         cudaStream_t s);
 cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s);
 

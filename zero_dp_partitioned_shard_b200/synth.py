@@ -55,6 +55,25 @@ def grads_f16(nd: int, n: int, seed: int, std: float = 1e-3, scale: float = 1.0,
     return out.view(np.uint16)
 
 
+def grads_bf16(nd: int, n: int, seed: int, std: float = 1e-3, scale: float = 1.0,
+               stride: int | None = None, pad_fill: float = float("nan")) -> np.ndarray:
+    """As ``grads_f16`` (same draws), rounded to bfloat16 instead: uint16 bits [nd, stride]."""
+    stride = n if stride is None else stride
+    assert stride >= n
+    out = torch.empty((nd, stride), dtype=torch.bfloat16)
+    for r in range(nd):
+        x = torch.randn(int(n), generator=_gen(seed * 1000003 + r), dtype=torch.float32)
+        out[r, :n] = (x * (std * scale)).to(torch.bfloat16)
+        out[r, n:] = pad_fill
+    return out.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 array -> bfloat16 bit patterns via torch's round-to-nearest-even cast."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
 def fp16_bits(x: np.ndarray) -> np.ndarray:
     """fp32 array -> fp16 bit patterns via numpy's round-to-nearest-even cast."""
     return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
