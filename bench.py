@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused ZeRO shard-step params/s and achieved HBM GB/s (fraction of B200 peak)"
 UNIT = "params/s"
+STORAGES = {"fp16": 0, "bf16": 1}   # the library's ZERO_STORAGE_* codes
 FALLBACK_HBM_GBS = 6650.0  # used only if MEASURED_PEAKS.json is absent
 
 
@@ -167,7 +168,7 @@ class ClockSampler:
 class Bench:
     """Device buffers and the C-ABI arguments of one workload on one GPU."""
 
-    def __init__(self, wl: dict, psi_override: int | None, seed: int):
+    def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0):
         import torch
         from zero_dp_partitioned_shard_b200 import binding as B
         from zero_dp_partitioned_shard_b200 import synth
@@ -189,17 +190,19 @@ class Bench:
         n_state = oc * L
         dev = torch.device("cuda")
         spec = wl["mode"] == B.ZERO_MODE_SPECULATIVE
+        self.storage = storage
+        h16 = torch.bfloat16 if storage == B.ZERO_STORAGE_BF16 else torch.float16
         # gradient contributions
         if wl["layout"] == B.ZERO_GRADS_FULL:
             stride = info.psi_pad
-            self.grads = torch.empty(self.nd * stride, dtype=torch.float16, device=dev)
+            self.grads = torch.empty(self.nd * stride, dtype=h16, device=dev)
             for r in range(self.nd):
                 row = self.grads[r * stride:(r + 1) * stride]
                 synth.fill_normal_(row[:psi], seed=seed * 1000 + r, std=1e-3, scale=wl["S"])
                 row[psi:].zero_()
         else:
             stride = L
-            self.grads = torch.empty(oc * self.nd * L, dtype=torch.float16, device=dev)
+            self.grads = torch.empty(oc * self.nd * L, dtype=h16, device=dev)
             synth.fill_normal_(self.grads, seed=seed * 1000, std=1e-3, scale=wl["S"])
         self.stride = stride
         self.grad_bytes = self.grads.numel() * 2
@@ -209,9 +212,10 @@ class Bench:
         self.exp_avg = [f32(), f32() if spec else None]
         self.exp_avg_sq = [f32(), f32() if spec else None]
         self.stash = f32() if wl["mode"] == B.ZERO_MODE_STASH else None
-        self.params = torch.zeros(psi, dtype=torch.float16, device=dev)
+        self.params = torch.zeros(psi, dtype=h16, device=dev)
         stream = torch.cuda.current_stream().cuda_stream
-        B.zero_cast_params(self.plan, self.master[0].data_ptr(), self.params.data_ptr(), o0, oc, stream)
+        B.zero_cast_params(self.plan, self.master[0].data_ptr(), self.params.data_ptr(), o0, oc, stream,
+                           storage=storage)
         self.opt_state = torch.zeros(B.OPT_STATE_BYTES, dtype=torch.uint8, device=dev)
         self.result = torch.zeros(B.RESULT_BYTES, dtype=torch.uint8, device=dev)
         B.zero_opt_state_init(self.opt_state.data_ptr(), stream)
@@ -224,13 +228,13 @@ class Bench:
             exp_avg=tuple(ptr(t) for t in self.exp_avg),
             exp_avg_sq=tuple(ptr(t) for t in self.exp_avg_sq), params=self.params.data_ptr(),
             grad_stash=ptr(self.stash), opt_state=self.opt_state.data_ptr(),
-            result=self.result.data_ptr())
+            result=self.result.data_ptr(), storage=storage)
         # stage-3 view: after its own update the rank assembles the full fp16
         # buffer from the other owners' (seeded) parameter shards
         self.shards, self.shard_ptrs, self.assembled = None, None, 0
         if wl.get("assemble"):
             others = [r for r in range(self.nd) if not (o0 <= r < o0 + oc)]
-            self.shards = torch.empty(len(others), L, dtype=torch.float16, device=dev)
+            self.shards = torch.empty(len(others), L, dtype=h16, device=dev)
             for k, r in enumerate(others):
                 synth.fill_normal_(self.shards[k], seed=seed * 1000 + 500 + r, std=0.02)
             self.shard_ptrs = [0] * self.nd
@@ -299,18 +303,23 @@ def _barrier(world: int):
         dist.barrier()
 
 
-def cpu_baseline(wl: dict, budget_s: float, sample_psi: int, threads: int) -> dict:
+def _draw_grads(storage: int):
+    from zero_dp_partitioned_shard_b200 import synth
+    return synth.grads_bf16 if storage == 1 else synth.grads_f16
+
+
+def cpu_baseline(wl: dict, budget_s: float, sample_psi: int, threads: int, storage: int = 0) -> dict:
     """The CPU oracle, as it stands, on a bounded sample of the workload."""
     import oracle
     from zero_dp_partitioned_shard_b200 import synth
     nd = wl["nd"]
-    G = synth.grads_f16(nd, sample_psi, seed=5, std=1e-3, scale=wl["S"])
+    G = _draw_grads(storage)(nd, sample_psi, seed=5, std=1e-3, scale=wl["S"])
     master = synth.normal_f32(sample_psi, seed=6, std=0.02)
     m = np.zeros(sample_psi, np.float32)
     v = np.zeros(sample_psi, np.float32)
     P = np.zeros(sample_psi, np.uint16)
     hp = oracle.HP(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
-                   loss_scale=wl["S"], max_grad_norm=wl["clip"])
+                   loss_scale=wl["S"], max_grad_norm=wl["clip"], storage=storage)
     opt = oracle.Opt()
     steps, t0 = 0, time.perf_counter()
     while True:
@@ -337,13 +346,14 @@ def run_reference(args, wl_name: str, wl: dict):
     threads = oracle.host_threads()
     nd = wl["nd"]
     sample = args.ref_sample
-    G = synth.grads_f16(nd, sample, seed=5, std=1e-3, scale=wl["S"])
+    storage = STORAGES[args.storage]
+    G = _draw_grads(storage)(nd, sample, seed=5, std=1e-3, scale=wl["S"])
     master = synth.normal_f32(sample, seed=6, std=0.02)
     m = np.zeros(sample, np.float32)
     v = np.zeros(sample, np.float32)
     P = np.zeros(sample, np.uint16)
     hp = oracle.HP(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
-                   loss_scale=wl["S"], max_grad_norm=wl["clip"])
+                   loss_scale=wl["S"], max_grad_norm=wl["clip"], storage=storage)
     opt = oracle.Opt()
     for _ in range(args.warmup):
         oracle.step(G, master, m, v, P, hp, opt, threads=threads)
@@ -358,7 +368,7 @@ def run_reference(args, wl_name: str, wl: dict):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": wl_name, "description": wl["desc"], "psi": _psi_of(wl),
-                   "nd": nd, "sample_params_per_step": sample},
+                   "nd": nd, "storage": args.storage, "sample_params_per_step": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{args.steps} steps over {sample:,} params x Nd={nd}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -449,6 +459,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gpt2-1.5b-stage2-nd8")
     ap.add_argument("--psi", type=int, default=0, help="smaller Psi of the same workload (profiling)")
+    ap.add_argument("--storage", choices=sorted(STORAGES), default="fp16",
+                    help="16-bit format of gradients and parameters")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -476,7 +488,7 @@ def main():
     import torch
     from zero_dp_partitioned_shard_b200 import binding as B
     world, rank, local = _dist()
-    bench = Bench(wl, args.psi or None, seed=1 + rank)
+    bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage])
     alg, moved = bytes_per_param(wl["nd"], wl["mode"])
 
     # --- device-resident timing ---
@@ -515,7 +527,7 @@ def main():
         import psutil
         need = bench.grad_bytes
         if psutil.virtual_memory().available > 2.5 * need:
-            g_host = torch.empty(bench.grads.numel(), dtype=torch.float16, pin_memory=True)
+            g_host = torch.empty(bench.grads.numel(), dtype=bench.grads.dtype, pin_memory=True)
             g_host.copy_(bench.grads)
             r_host = torch.empty(B.RESULT_BYTES, dtype=torch.uint8, pin_memory=True)
             torch.cuda.synchronize()
@@ -549,7 +561,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": args.workload, "description": wl["desc"], "psi": bench.psi,
-                   "nd": wl["nd"], "stage": wl["stage"], "owned_params_per_gpu": bench.owned,
+                   "nd": wl["nd"], "stage": wl["stage"], "storage": args.storage,
+                   "owned_params_per_gpu": bench.owned,
                    "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
                    "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
                    "assembled_params": bench.assembled,
@@ -571,7 +584,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.cpu_sample,
-                                            oracle.host_threads())
+                                            oracle.host_threads(), STORAGES[args.storage])
     bench.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
