@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 4
+#define ZERO_SHARD_ABI_VERSION 5
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -254,7 +254,11 @@ typedef struct zero_hparams {
  *     256-byte aligned; contents need no initialisation and are clobbered.
  *   timing_events: optional pair of cudaEvent_t (as void*) recorded on the
  *     stream immediately before and after the parameter-update kernel(s), so
- *     a caller can time the dominant kernel alone; NULL entries = none. */
+ *     a caller can time the dominant kernel alone; NULL entries = none.
+ *   peers: NULL, or the peer tables of the fused reduce-scatter + update +
+ *     all-gather (zero_peer_args below); grads and grad_rank_stride are then
+ *     ignored. */
+typedef struct zero_peer_args zero_peer_args;
 typedef struct zero_step_args {
     const void* grads;
     int64_t grad_rank_stride;
@@ -272,7 +276,67 @@ typedef struct zero_step_args {
     void* workspace;
     size_t workspace_bytes;
     void* timing_events[2];
+    const zero_peer_args* peers;   /* host pointer, may be NULL */
 } zero_step_args;
+
+/* ---- fused reduce-scatter + update + all-gather over peer memory ------------- */
+/* With one process per GPU, a step reads every rank's contribution to its own
+ * shard (the reduce-scatter) and ends with every rank holding every owner's
+ * new 16-bit parameters (the all-gather) -- "ZeRO: partitioning training
+ * state across GPUs" (upskillscore.com), "How it works"; "ZeRO memory
+ * optimization" (trishampatil.com), the figure under "Forward/Backward Under
+ * ZeRO-3".  With peer tables the step's kernels do both themselves, in the
+ * same pass as the arithmetic: they load rank r's contribution straight from
+ * rank_grads[r] (this GPU's memory or another GPU's, mapped into this
+ * process with zero_ipc_open) and store each new parameter into params and
+ * into every param_dests[d] (the other ranks' full parameter buffers).
+ * Nothing waits on another GPU inside a kernel: the caller orders the ranks
+ * with stream-ordered collectives -- one after the gradients are written and
+ * before zero_shard_step_begin (every contribution is complete), the vote
+ * all-reduce between begin and end, and one after end (every rank's
+ * parameters are complete and its gradient buffer is free again).
+ *   rank_grads[r], r < nd: device, rank r's 16-bit gradient buffer in the
+ *     FULL layout (the element at flat index f at [f]); the call reads
+ *     [o * L, o * L + real_len_o) of it for each owner o of the call.
+ *   param_dests[d], d < n_param_dests: device, full parameter buffers (psi
+ *     elements, the all-gather layout) written like params.
+ *   Entries past nd / n_param_dests are ignored.  The arithmetic and the
+ *   results are exactly those of the strided call with the same data.
+ * Errors (besides zero_shard_step's): UNSUPPORTED if nd > ZERO_MAX_PEERS or
+ * grad_layout is PER_OWNER; INVALID_ARG for a NULL entry or n_param_dests
+ * outside [0, ZERO_MAX_PEERS]; ALIGNMENT for an entry not 2-byte aligned
+ * (16-byte aligned entries keep the vectorised path). */
+#define ZERO_MAX_PEERS 64
+struct zero_peer_args {
+    const void* rank_grads[ZERO_MAX_PEERS];
+    void* param_dests[ZERO_MAX_PEERS];
+    int32_t n_param_dests;
+    int32_t reserved;        /* must be 0 */
+};
+
+/* A device buffer exported for mapping into another process (CUDA IPC).
+ * handle: the cudaIpcMemHandle_t of the allocation that holds the buffer;
+ * offset: the buffer's byte offset inside that allocation. */
+typedef struct zero_ipc_handle {
+    unsigned char handle[64];
+    int64_t offset;
+    int32_t device;          /* ordinal of the exporting device */
+    int32_t reserved;
+} zero_ipc_handle;
+
+/* Exports the device buffer at dev_ptr (anywhere inside a cudaMalloc
+ * allocation) into *out.  Errors: INVALID_ARG for a null argument or a
+ * pointer that is not device memory; CUDA. */
+ZERO_API zero_status zero_ipc_export(const void* dev_ptr, zero_ipc_handle* out);
+/* Maps a buffer exported by another process into this one, with peer access
+ * enabled when it lives on another GPU, and returns its address in *dev_ptr.
+ * Mapping the same allocation again reuses the mapping (reference counted).
+ * Errors: INVALID_ARG; CUDA (e.g. a handle exported by this same process,
+ * which CUDA refuses to open). */
+ZERO_API zero_status zero_ipc_open(const zero_ipc_handle* h, void** dev_ptr);
+/* Releases a mapping made by zero_ipc_open (the address it returned).
+ * Errors: INVALID_ARG for an address zero_ipc_open did not return; CUDA. */
+ZERO_API zero_status zero_ipc_close(void* dev_ptr);
 
 /* Writes {t = 0, beta1_pow = beta2_pow = 1, skipped = 0, cur = 0, static
  * loss scaling} into the device zero_opt_state at opt_state, on stream. */

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
     lib = B.lib()
     for name in declared:
         assert getattr(lib, name) is not None
-    assert B.zero_abi_version() == 4
+    assert B.zero_abi_version() == 5
     # nothing else leaks out of the library (hidden visibility)
     assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
 
@@ -60,6 +60,8 @@ int main(void) {
   O(zero_step_args, timing_events) O(zero_hparams, mode) O(zero_opt_state, cur)
   O(zero_step_result, overflow) O(zero_step_result, status) O(zero_step_result, loss_scale)
   O(zero_opt_state, loss_scale) O(zero_opt_state, growth_interval) O(zero_plan_desc, nd) O(zero_plan_info, nd)
+  S(zero_peer_args) S(zero_ipc_handle) O(zero_step_args, peers) O(zero_peer_args, param_dests)
+  O(zero_peer_args, n_param_dests) O(zero_ipc_handle, offset) O(zero_ipc_handle, device)
   return 0;
 }
 """
@@ -76,7 +78,8 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
     got = {k: int(v) for k, v in got.items()}
     py = {"zero_plan_desc": B.PlanDesc, "zero_plan_info": B.PlanInfo, "zero_segment": B.Segment,
           "zero_state_report": B.StateReport, "zero_opt_state": B.OptState,
-          "zero_step_result": B.StepResult, "zero_hparams": B.HParams, "zero_step_args": B.StepArgs}
+          "zero_step_result": B.StepResult, "zero_hparams": B.HParams, "zero_step_args": B.StepArgs,
+          "zero_peer_args": B.PeerArgs, "zero_ipc_handle": B.IpcHandle}
     for cname, ctype in py.items():
         assert got[cname] == C.sizeof(ctype), cname
     for key, val in got.items():
@@ -175,6 +178,10 @@ def _args(**kw):
     ("misaligned_params", B.ZERO_ERR_ALIGNMENT), ("small_ws", B.ZERO_ERR_WORKSPACE),
     ("null_ws", B.ZERO_ERR_WORKSPACE), ("misaligned_ws", B.ZERO_ERR_ALIGNMENT),
     ("reserved", B.ZERO_ERR_INVALID_ARG), ("bad_storage", B.ZERO_ERR_INVALID_ARG),
+    ("peer_layout", B.ZERO_ERR_UNSUPPORTED), ("peer_null_grad", B.ZERO_ERR_INVALID_ARG),
+    ("peer_misaligned_grad", B.ZERO_ERR_ALIGNMENT), ("peer_null_dest", B.ZERO_ERR_INVALID_ARG),
+    ("peer_misaligned_dest", B.ZERO_ERR_ALIGNMENT), ("peer_n_dests", B.ZERO_ERR_INVALID_ARG),
+    ("peer_reserved", B.ZERO_ERR_INVALID_ARG),
 ])
 def test_step_validation_rejects_before_launch(case, status):
     plan = B.zero_plan(1000, 4, stage=1, align_elems=8)
@@ -217,6 +224,26 @@ def test_step_validation_rejects_before_launch(case, status):
     elif case == "bad_storage":
         args = _args()
         args.storage = 2
+    elif case.startswith("peer_"):
+        grads = [FAKE + (r << 20) for r in range(4)]
+        dests = [FAKE + (9 << 20), FAKE + (10 << 20)]
+        layout = B.ZERO_GRADS_FULL
+        if case == "peer_layout":
+            layout = B.ZERO_GRADS_PER_OWNER
+        elif case == "peer_null_grad":
+            grads[2] = 0
+        elif case == "peer_misaligned_grad":
+            grads[1] += 1
+        elif case == "peer_null_dest":
+            dests[1] = 0
+        elif case == "peer_misaligned_dest":
+            dests[0] += 3
+        q = B.peer_args(grads, dests)
+        if case == "peer_n_dests":
+            q.n_param_dests = B.ZERO_MAX_PEERS + 1
+        elif case == "peer_reserved":
+            q.reserved = 1
+        args = B.attach_peers(_args(grads=0, grad_layout=layout), q)
     before = B.zero_launch_count()
     try:
         with pytest.raises(B.ZeroError) as e:
@@ -226,6 +253,44 @@ def test_step_validation_rejects_before_launch(case, status):
     finally:
         B.zero_plan_destroy(plan)
     assert B.zero_launch_count() == before
+
+
+def test_peer_tables_replace_the_strided_gradients():
+    """With peer tables the gradient pointer and stride are not used; a plan
+    with more ranks than the tables hold is refused."""
+    plan = B.zero_plan(1000, 4, stage=2, align_elems=8)
+    try:
+        q = B.peer_args([FAKE + (r << 20) for r in range(4)], [FAKE + (7 << 20)])
+        args = B.attach_peers(_args(grads=0, grad_rank_stride=0), q)
+        assert B.zero_workspace_bytes(plan, B.hparams(loss_scale=1.0), args) == 256
+        B.attach_peers(args, None)
+        with pytest.raises(B.ZeroError) as e:     # without the tables the null grads are an error
+            B.zero_workspace_bytes(plan, B.hparams(loss_scale=1.0), args)
+        assert e.value.status == B.ZERO_ERR_INVALID_ARG
+    finally:
+        B.zero_plan_destroy(plan)
+    big = B.zero_plan(100_000, B.ZERO_MAX_PEERS + 1, stage=2, align_elems=8)
+    try:
+        q = B.peer_args([FAKE] * B.ZERO_MAX_PEERS)
+        args = B.attach_peers(_args(grads=0, owner_count=1), q)
+        with pytest.raises(B.ZeroError) as e:
+            B.zero_workspace_bytes(big, B.hparams(loss_scale=1.0), args)
+        assert e.value.status == B.ZERO_ERR_UNSUPPORTED
+    finally:
+        B.zero_plan_destroy(big)
+
+
+def test_ipc_helpers_validate_arguments():
+    lib = B.lib()
+    assert lib.zero_ipc_export(None, None) == B.ZERO_ERR_INVALID_ARG
+    assert lib.zero_ipc_open(None, None) == B.ZERO_ERR_INVALID_ARG
+    with pytest.raises(B.ZeroError) as e:   # not an address zero_ipc_open returned
+        B.zero_ipc_close(FAKE)
+    assert e.value.status == B.ZERO_ERR_INVALID_ARG
+    h = B.IpcHandle()
+    h.offset = -1
+    p = C.c_void_p()
+    assert lib.zero_ipc_open(C.byref(h), C.byref(p)) == B.ZERO_ERR_INVALID_ARG
 
 
 def test_workspace_bytes_per_mode():

@@ -119,3 +119,56 @@ def test_gloo_protocol_matches_single_process_oracle(world, inject, clip):
     assert np.array_equal(got_master.view(np.uint32), ref_master.view(np.uint32))
     for r in results:   # every process holds the same, complete parameter buffer
         assert np.array_equal(r[5], ref_P)
+
+
+def _tables_worker(rank, world, port, out):
+    """Host side of the fused peer step: the IPC exports travel in rank order
+    and become one gradient table (this process's own buffer at its rank) and
+    the other ranks' parameter buffers as destinations."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from zero_dp_partitioned_shard_b200 import distributed as D
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        mine = (f"grad-export-{rank}".encode(), f"param-export-{rank}".encode())
+        handles = D.exchange_handles(mine)
+        opened_here = []
+
+        def opener(h):        # stands in for zero_ipc_open: a distinct address per export
+            opened_here.append(h)
+            return 1_000_000 + int(h.decode().rsplit("-", 1)[1]) * 10 + (1 if h.startswith(b"param") else 0)
+
+        own = (7, 8)
+        grads, dests, opened = D.peer_tables(handles, rank, own, opener)
+        vote = torch.tensor([float(rank + 1), 1.0 if rank == world - 1 else 0.0], dtype=torch.float64)
+        D.reduce_vote(vote)
+        out.put((rank, handles, grads, dests, opened, opened_here, vote.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_peer_tables_from_exchanged_exports(world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_tables_worker, args=(r, world, port, out)) for r in range(world)]
+    for pr in procs:
+        pr.start()
+    got = sorted([out.get(timeout=120) for _ in range(world)], key=lambda x: x[0])
+    for pr in procs:
+        pr.join(timeout=60)
+        assert pr.exitcode == 0
+    for rank, handles, grads, dests, opened, opened_here, vote in got:
+        assert [h[0] for h in handles] == [f"grad-export-{r}".encode() for r in range(world)]
+        assert grads[rank] == 7                       # own gradient: not mapped, the local address
+        others = [r for r in range(world) if r != rank]
+        assert [grads[r] for r in others] == [1_000_000 + r * 10 for r in others]
+        assert dests == [1_000_000 + r * 10 + 1 for r in others]   # other ranks' parameters, rank order
+        assert sorted(opened) == sorted([1_000_000 + r * 10 for r in others] + dests)
+        assert len(opened_here) == 2 * (world - 1)    # nothing of its own is mapped
+        assert vote == [world * (world + 1) / 2, 1.0]

@@ -36,6 +36,8 @@ ZERO_GRADS_PER_OWNER = 1
 ZERO_STORAGE_FP16 = 0
 ZERO_STORAGE_BF16 = 1
 
+ZERO_MAX_PEERS = 64
+
 ZERO_STATIC_SCRATCH_BYTES = 1 << 20  # static scratch of zero_shard_step_static_scratch
 ZERO_VOTE_OFFSET = 128               # byte offset of the split step's fp64[2] vote in the workspace
 
@@ -104,7 +106,18 @@ class StepArgs(C.Structure):
                 ("exp_avg_sq", C.c_void_p * 2), ("params", C.c_void_p),
                 ("grad_stash", C.c_void_p), ("opt_state", C.c_void_p), ("result", C.c_void_p),
                 ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
-                ("timing_events", C.c_void_p * 2)]
+                ("timing_events", C.c_void_p * 2), ("peers", C.c_void_p)]
+
+
+class PeerArgs(C.Structure):
+    _fields_ = [("rank_grads", C.c_void_p * ZERO_MAX_PEERS),
+                ("param_dests", C.c_void_p * ZERO_MAX_PEERS),
+                ("n_param_dests", C.c_int32), ("reserved", C.c_int32)]
+
+
+class IpcHandle(C.Structure):
+    _fields_ = [("handle", C.c_ubyte * 64), ("offset", C.c_int64), ("device", C.c_int32),
+                ("reserved", C.c_int32)]
 
 
 _lib = None
@@ -130,6 +143,9 @@ SIGNATURES = {
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
     "zero_gather_tensors": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, C.c_int32, _P]),
+    "zero_ipc_export": (_S, [_P, C.POINTER(IpcHandle)]),
+    "zero_ipc_open": (_S, [C.POINTER(IpcHandle), C.POINTER(_P)]),
+    "zero_ipc_close": (_S, [_P]),
     "zero_abi_version": (C.c_int32, []),
     "zero_strerror": (C.c_char_p, [_S]),
     "zero_last_error": (C.c_char_p, []),
@@ -151,7 +167,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 4:
+        if L.zero_abi_version() != 5:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -278,6 +294,25 @@ def zero_cast_params(plan: int, master: int, params: int, owner_first: int, owne
            "zero_cast_params")
 
 
+def zero_ipc_export(dev_ptr: int) -> bytes:
+    """The CUDA IPC export of a device buffer, as bytes to send to other processes."""
+    h = IpcHandle()
+    _check(lib().zero_ipc_export(dev_ptr, C.byref(h)), "zero_ipc_export")
+    return bytes(h)
+
+
+def zero_ipc_open(handle: bytes) -> int:
+    """Maps a buffer exported by another process; returns its address here."""
+    h = IpcHandle.from_buffer_copy(handle)
+    p = C.c_void_p()
+    _check(lib().zero_ipc_open(C.byref(h), C.byref(p)), "zero_ipc_open")
+    return p.value
+
+
+def zero_ipc_close(dev_ptr: int) -> None:
+    _check(lib().zero_ipc_close(dev_ptr), "zero_ipc_close")
+
+
 def zero_abi_version() -> int:
     return lib().zero_abi_version()
 
@@ -334,6 +369,27 @@ def step_args(*, grads: int, grad_rank_stride: int, master, exp_avg, exp_avg_sq,
     a.workspace = workspace or None
     a.workspace_bytes = workspace_bytes
     return a
+
+
+def peer_args(rank_grads, param_dests=()) -> PeerArgs:
+    """Peer tables: rank_grads[r] = rank r's gradient buffer, param_dests = the
+    other full parameter buffers that receive every new parameter."""
+    if len(rank_grads) > ZERO_MAX_PEERS or len(param_dests) > ZERO_MAX_PEERS:
+        raise ValueError(f"at most {ZERO_MAX_PEERS} ranks and destinations")
+    q = PeerArgs()
+    for r, g in enumerate(rank_grads):
+        q.rank_grads[r] = g or None
+    for d, p in enumerate(param_dests):
+        q.param_dests[d] = p or None
+    q.n_param_dests = len(param_dests)
+    return q
+
+
+def attach_peers(args: StepArgs, peers: PeerArgs | None) -> StepArgs:
+    """Points args at the peer tables (None detaches them); args keeps them alive."""
+    args._peers_ref = peers
+    args.peers = C.cast(C.pointer(peers), C.c_void_p) if peers is not None else None
+    return args
 
 
 def opt_state_from_bytes(raw: bytes) -> OptState:

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libzero_shard.so")
 
-SOURCES = ["kernels.cu", "api.cpp", "plan.cpp", "static_scratch.cu"]
+SOURCES = ["kernels.cu", "api.cpp", "plan.cpp", "static_scratch.cu", "peer.cpp"]
 HEADERS = [os.path.join(CSRC, "zs_internal.h"), os.path.join(INCLUDE, "zero_shard.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

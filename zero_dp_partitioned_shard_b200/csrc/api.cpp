@@ -64,6 +64,8 @@ bool segs_vec_ok(const std::vector<zs::SegList>& lists)
 
 int64_t effective_stride(const zero_plan_s& p, const zero_step_args& a)
 {
+    if (a.peers) // one buffer per rank: the stride is not used
+        return 0;
     if (a.grad_layout == ZERO_GRADS_PER_OWNER && a.grad_rank_stride == 0)
         return p.shard_len;
     return a.grad_rank_stride;
@@ -96,14 +98,38 @@ zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_st
                     a->owner_first, a->owner_first, a->owner_count, p->nd);
     if (a->grad_layout != ZERO_GRADS_FULL && a->grad_layout != ZERO_GRADS_PER_OWNER)
         return fail(ZERO_ERR_INVALID_ARG, "unknown grad_layout %d", a->grad_layout);
+    if (a->peers) {
+        const zero_peer_args& q = *a->peers;
+        if (a->grad_layout != ZERO_GRADS_FULL)
+            return fail(ZERO_ERR_UNSUPPORTED, "peer tables need the FULL gradient layout");
+        if (p->nd > ZERO_MAX_PEERS)
+            return fail(ZERO_ERR_UNSUPPORTED, "peer tables hold at most %d ranks (nd = %d)", ZERO_MAX_PEERS, p->nd);
+        if (q.n_param_dests < 0 || q.n_param_dests > ZERO_MAX_PEERS)
+            return fail(ZERO_ERR_INVALID_ARG, "n_param_dests %d outside [0, %d]", q.n_param_dests, ZERO_MAX_PEERS);
+        if (q.reserved != 0)
+            return fail(ZERO_ERR_INVALID_ARG, "reserved fields must be 0");
+        for (int r = 0; r < p->nd; ++r) {
+            if (!q.rank_grads[r])
+                return fail(ZERO_ERR_INVALID_ARG, "rank_grads[%d] is null", r);
+            if (!aligned(q.rank_grads[r], 2))
+                return fail(ZERO_ERR_ALIGNMENT, "rank_grads[%d] must be 2-byte aligned", r);
+        }
+        for (int d = 0; d < q.n_param_dests; ++d) {
+            if (!q.param_dests[d])
+                return fail(ZERO_ERR_INVALID_ARG, "param_dests[%d] is null", d);
+            if (!aligned(q.param_dests[d], 2))
+                return fail(ZERO_ERR_ALIGNMENT, "param_dests[%d] must be 2-byte aligned", d);
+        }
+    }
     const int64_t stride = effective_stride(*p, *a);
-    if (a->grad_layout == ZERO_GRADS_FULL && p->nd > 1 && stride < p->psi)
+    if (!a->peers && a->grad_layout == ZERO_GRADS_FULL && p->nd > 1 && stride < p->psi)
         return fail(ZERO_ERR_INVALID_ARG, "FULL layout needs grad_rank_stride >= psi (%lld < %lld)",
                     (long long)stride, (long long)p->psi);
     if (a->grad_layout == ZERO_GRADS_PER_OWNER && stride < p->shard_len)
         return fail(ZERO_ERR_INVALID_ARG, "PER_OWNER layout needs grad_rank_stride >= L (%lld < %lld)",
                     (long long)stride, (long long)p->shard_len);
-    if (!a->grads || !a->master[0] || !a->exp_avg[0] || !a->exp_avg_sq[0] || !a->params || !a->opt_state)
+    if ((!a->grads && !a->peers) || !a->master[0] || !a->exp_avg[0] || !a->exp_avg_sq[0] || !a->params ||
+        !a->opt_state)
         return fail(ZERO_ERR_INVALID_ARG, "null device buffer (grads, master, exp_avg, exp_avg_sq, params, opt_state)");
     const bool spec = hp->mode == ZERO_MODE_SPECULATIVE;
     if (spec && (!a->master[1] || !a->exp_avg[1] || !a->exp_avg_sq[1]))
@@ -152,8 +178,15 @@ LaunchPlan plan_launches(const zero_plan_s& p, const zero_hparams& hp, const zer
         lp.whole.push_back(empty);
     }
     const bool spec = hp.mode == ZERO_MODE_SPECULATIVE;
-    bool vec = (L % 8 == 0) && (p.bucket % 8 == 0) && (stride % 8 == 0) && aligned(a.grads, 16) &&
-               aligned(a.params, 16);
+    bool vec = (L % 8 == 0) && (p.bucket % 8 == 0) && (stride % 8 == 0) && aligned(a.params, 16);
+    if (a.peers) {
+        for (int r = 0; r < p.nd; ++r)
+            vec = vec && aligned(a.peers->rank_grads[r], 16);
+        for (int d = 0; d < a.peers->n_param_dests; ++d)
+            vec = vec && aligned(a.peers->param_dests[d], 16);
+    } else {
+        vec = vec && aligned(a.grads, 16);
+    }
     for (int k = 0; k < (spec ? 2 : 1); ++k)
         vec = vec && aligned(a.master[k], 16) && aligned(a.exp_avg[k], 16) && aligned(a.exp_avg_sq[k], 16);
     if (hp.mode == ZERO_MODE_STASH)
@@ -285,6 +318,19 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
     u.one_minus_beta1 = 1.0f - h.beta1;
     u.one_minus_beta2 = 1.0f - h.beta2;
 
+    // peer tables: one gradient buffer per rank, extra parameter destinations
+    zs::PeerTable peer_table;
+    const zs::PeerTable* peers = nullptr;
+    if (a.peers) {
+        std::memset(&peer_table, 0, sizeof peer_table);
+        for (int r = 0; r < p.nd; ++r)
+            peer_table.grads[r] = static_cast<const uint16_t*>(a.peers->rank_grads[r]);
+        for (int d = 0; d < a.peers->n_param_dests; ++d)
+            peer_table.dests[d] = static_cast<uint16_t*>(a.peers->param_dests[d]);
+        peer_table.n_dests = a.peers->n_param_dests;
+        peers = &peer_table;
+    }
+
     const bool spec = h.mode == ZERO_MODE_SPECULATIVE;
     const bool first_half = phase != PHASE_END;
     const bool second_half = phase != PHASE_BEGIN;
@@ -299,7 +345,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
                 return cuda_fail(e, "timing event");
             for (const auto& b : lp.buckets)
                 for (const auto& l : b)
-                    if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, str)) != cudaSuccess)
+                    if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, peers, str)) != cudaSuccess)
                         return cuda_fail(e, "update launch");
             if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
                 return cuda_fail(e, "timing event");
@@ -311,7 +357,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
                 (e = zs::launch_vote_apply(ws, true, h.max_grad_norm, st, res, str)) != cudaSuccess)
                 return cuda_fail(e, "vote launch");
             for (size_t i = 0; i < lp.whole.size(); ++i)
-                if ((e = zs::launch_commit(lp.vec, u, lp.whole[i], i == 0, st, res, str)) != cudaSuccess)
+                if ((e = zs::launch_commit(lp.vec, u, lp.whole[i], i == 0, st, res, peers, str)) != cudaSuccess)
                     return cuda_fail(e, "commit launch");
         }
         return ZERO_OK;
@@ -332,7 +378,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
         for (const auto& b : lp.buckets) {
             for (const auto& l : b) {
                 sa.partials = partials + n_partials;
-                if ((e = zs::launch_stats(lp.vec, sa, l, str)) != cudaSuccess)
+                if ((e = zs::launch_stats(lp.vec, sa, l, peers, str)) != cudaSuccess)
                     return cuda_fail(e, "statistics launch");
                 n_partials += zs::stats_blocks(lp.vec, l);
             }
@@ -352,7 +398,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
         if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
             return cuda_fail(e, "timing event");
         for (const auto& l : lp.whole)
-            if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, str)) != cudaSuccess)
+            if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, peers, str)) != cudaSuccess)
                 return cuda_fail(e, "update launch");
         if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
             return cuda_fail(e, "timing event");

@@ -16,7 +16,11 @@
 //     fixed shuffle pattern and summed in a fixed order by a one-block kernel,
 //     so results are bit-reproducible for a given launch geometry.
 // No kernel waits on another block, a flag or a peer: ordering between the
-// kernels of a step is plain stream order.
+// kernels of a step is plain stream order.  With peer tables the same kernels
+// load the contributions from each rank's own buffer (possibly another GPU's
+// memory) and store every new parameter into each rank's parameter buffer:
+// the reduce-scatter and the all-gather ride on the update's own loads and
+// stores.
 //
 // Arithmetic per parameter (ZeRO leaves the optimizer's maths unchanged; the
 // pages name Adam with fp32 master, momentum and variance -- "ZeRO memory
@@ -31,6 +35,7 @@
 
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <unordered_map>
 #include <utility>
 
@@ -134,17 +139,66 @@ __device__ __forceinline__ uint16_t f2h(float f)
     return BF ? __bfloat16_as_ushort(__float2bfloat16_rn(f)) : __half_as_ushort(__float2half_rn(f));
 }
 
+// Where rank r's contributions to a run of elements start: the rank buffers
+// side by side at a fixed stride (one process holding the whole group), or one
+// buffer per rank through the peer table (each possibly another GPU's memory,
+// reached by plain loads over NVLink).
+struct StridedRanks {
+    const uint16_t* g;
+    int64_t rstride;
+    __device__ __forceinline__ const uint16_t* at(int r) const { return g + (int64_t)r * rstride; }
+};
+
+struct TableRanks {
+    const uint16_t* const* tbl;
+    int64_t off;
+    __device__ __forceinline__ const uint16_t* at(int r) const { return tbl[r] + off; }
+};
+
+struct NoPeers {};
+template <bool PEER>
+using PeerParam = typename std::conditional<PEER, PeerTable, NoPeers>::type;
+
+template <bool PEER>
+__device__ __forceinline__ auto ranks_at(const uint16_t* grads, const PeerParam<PEER>& pt, const Seg& sg, int64_t e)
+{
+    if constexpr (PEER)
+        return TableRanks{pt.grads, sg.g_off + e};
+    else
+        return StridedRanks{grads + sg.g_off + e, sg.g_rstride};
+}
+
+// New parameters go to params and, with peer tables, to every other rank's
+// parameter buffer as well (the all-gather as stores).
+template <bool PEER>
+__device__ __forceinline__ void store_params8(uint16_t* params, const PeerParam<PEER>& pt, int64_t off, uint4 v)
+{
+    __stcs(reinterpret_cast<uint4*>(params + off), v);
+    if constexpr (PEER)
+        for (int d = 0; d < pt.n_dests; ++d)
+            __stcs(reinterpret_cast<uint4*>(pt.dests[d] + off), v);
+}
+
+template <bool PEER>
+__device__ __forceinline__ void store_param1(uint16_t* params, const PeerParam<PEER>& pt, int64_t off, uint16_t v)
+{
+    params[off] = v;
+    if constexpr (PEER)
+        for (int d = 0; d < pt.n_dests; ++d)
+            pt.dests[d][off] = v;
+}
+
 // Rank-order sum of the Nd contributions of 8 consecutive parameters: the
 // loads of each group of 8 ranks are issued together, then added in order.
-template <bool BF>
-__device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, int nd, float s[8])
+template <bool BF, class Ranks>
+__device__ __forceinline__ void rank_sum8(const Ranks& rk, int nd, float s[8])
 {
     {
         uint4 x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
             if (u < nd)
-                x[u] = ld_stream(g + u * rstride);
+                x[u] = ld_stream(rk.at(u));
         unpack_h8<BF>(x[0], s);
 #pragma unroll
         for (int u = 1; u < 8; ++u) {
@@ -162,7 +216,7 @@ __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, in
 #pragma unroll
         for (int u = 0; u < 8; ++u)
             if (r + u < nd)
-                x[u] = ld_stream(g + (int64_t)(r + u) * rstride);
+                x[u] = ld_stream(rk.at(r + u));
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             if (r + u < nd) {
@@ -176,12 +230,12 @@ __device__ __forceinline__ void rank_sum8(const uint16_t* g, int64_t rstride, in
     }
 }
 
-template <bool BF>
-__device__ __forceinline__ float rank_sum1(const uint16_t* g, int64_t rstride, int nd)
+template <bool BF, class Ranks>
+__device__ __forceinline__ float rank_sum1(const Ranks& rk, int nd)
 {
-    float s = h2f<BF>(g[0]);
+    float s = h2f<BF>(rk.at(0)[0]);
     for (int r = 1; r < nd; ++r)
-        s = __fadd_rn(s, h2f<BF>(g[(int64_t)r * rstride]));
+        s = __fadd_rn(s, h2f<BF>(rk.at(r)[0]));
     return s;
 }
 
@@ -325,29 +379,30 @@ __global__ void zs_prep_kernel(const zero_opt_state* st, WsHeader* ws, float bet
 
 // One element, scalar loads and stores; returns true if its gradient is not
 // finite (only meaningful when the reduced gradient is computed here).
-template <int SRC, bool BF>
-__device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const Seg& sg, int64_t e, const AdamK& k,
-                                              float inv, const float* p_in, const float* m_in,
-                                              const float* v_in, float* p_out, float* m_out, float* v_out)
+template <int SRC, bool BF, bool PEER>
+__device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const PeerParam<PEER>& pt, const Seg& sg,
+                                              int64_t e, const AdamK& k, float inv, const float* p_in,
+                                              const float* m_in, const float* v_in, float* p_out, float* m_out,
+                                              float* v_out)
 {
     const int64_t so = sg.s_off + e;
     float g;
     if (SRC == kSrcStash)
         g = a.stash[so];
     else
-        g = __fmul_rn(rank_sum1<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
+        g = __fmul_rn(rank_sum1<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd), inv);
     float p = p_in[so], m = m_in[so], v = v_in[so];
     adam_update(__fmul_rn(g, k.clip), p, m, v, k);
     p_out[so] = p;
     m_out[so] = m;
     v_out[so] = v;
-    a.params[sg.p_off + e] = f2h<BF>(p);
+    store_param1<PEER>(a.params, pt, sg.p_off + e, f2h<BF>(p));
     return !isfinite(g);
 }
 
-template <int SRC, bool VEC, bool BF>
+template <int SRC, bool VEC, bool BF, bool PEER>
 __global__ void __launch_bounds__(kThreads, 2)
-zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
+zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, const __grid_constant__ PeerParam<PEER> pt)
 {
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
     wait_for_predecessor(); // bias corrections, slot, skip and clip come from the kernels before
@@ -380,7 +435,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             if (SRC == kSrcStash) {
                 ld_f8(a.stash + so, g);
             } else {
-                rank_sum8<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+                rank_sum8<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd, g);
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
                     g[q] = __fmul_rn(g[q], inv);
@@ -396,10 +451,10 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs)
             st_f8(p_out + so, p);
             st_f8(m_out + so, m);
             st_f8(v_out + so, v);
-            __stcs(reinterpret_cast<uint4*>(a.params + sg.p_off + e), pack_h8<BF>(p));
+            store_params8<PEER>(a.params, pt, sg.p_off + e, pack_h8<BF>(p));
         },
         [&](const Seg& sg, int64_t e) {
-            bad |= update_scalar<SRC, BF>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
+            bad |= update_scalar<SRC, BF, PEER>(a, pt, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
         });
     if (kSpec)
         flag_nonfinite(bad, &a.ws->overflow);
@@ -558,9 +613,10 @@ __device__ __forceinline__ int tile_segment(const int64_t* first_tile, int count
     return s;
 }
 
-template <int SRC, int EPT, bool BF>
+template <int SRC, int EPT, bool BF, bool PEER>
 __global__ void __launch_bounds__(kPipeThreads, 2)
-zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages)
+zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages,
+                      const __grid_constant__ PeerParam<PEER> pt)
 {
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
     constexpr int T = kPipeConsumers * EPT; // elements per tile
@@ -638,8 +694,8 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                     bulk_load(buf + T * 12, a.stash + so, n * 4, &full[st]);
                 } else {
                     const int r = j - 3;
-                    bulk_load(buf + T * 12 + r * (T * 2), a.grads + sg.g_off + e0 + (int64_t)r * sg.g_rstride,
-                              n * 2, &full[st]);
+                    bulk_load(buf + T * 12 + r * (T * 2), ranks_at<PEER>(a.grads, pt, sg, e0).at(r), n * 2,
+                              &full[st]);
                 }
             }
         }
@@ -708,6 +764,9 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 stg_f<EPT>(m_out + so, m);
                 stg_f<EPT>(v_out + so, v);
                 stg_h<EPT, BF>(a.params + sg.p_off + e0 + i0, p);
+                if constexpr (PEER)
+                    for (int d = 0; d < pt.n_dests; ++d)
+                        stg_h<EPT, BF>(pt.dests[d] + sg.p_off + e0 + i0, p);
             }
             __syncwarp();
             if (lane == 0)
@@ -720,7 +779,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 const Seg& sg = segs.seg[si];
                 const int64_t e = (sg.n >> 3) * 8 + gtid;
                 if (e < sg.n)
-                    bad |= update_scalar<SRC, BF>(a, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
+                    bad |= update_scalar<SRC, BF, PEER>(a, pt, sg, e, k, inv, p_in, m_in, v_in, p_out, m_out, v_out);
             }
         }
         if (kSpec)
@@ -738,9 +797,9 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
 //     optionally the fp32 reduced gradient (stash)
 // ---------------------------------------------------------------------------
 
-template <bool VEC, bool STASH, bool BF>
+template <bool VEC, bool STASH, bool BF, bool PEER>
 __global__ void __launch_bounds__(kThreads, 2)
-zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
+zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs, const __grid_constant__ PeerParam<PEER> pt)
 {
     // The buckets of a step are independent: the next statistics launch may
     // start as soon as this one is resident.  Each launch waits for its
@@ -757,7 +816,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
         segs,
         [&](const Seg& sg, int64_t e) {
             float g[8];
-            rank_sum8<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd, g);
+            rank_sum8<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd, g);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 g[q] = __fmul_rn(g[q], inv);
@@ -769,7 +828,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs)
                 st_f8(a.stash + sg.s_off + e, g);
         },
         [&](const Seg& sg, int64_t e) {
-            const float g = __fmul_rn(rank_sum1<BF>(a.grads + sg.g_off + e, sg.g_rstride, a.nd), inv);
+            const float g = __fmul_rn(rank_sum1<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd), inv);
             bad |= !isfinite(g);
             const double d = (double)g;
             acc = __dadd_rn(acc, __dmul_rn(d, d));
@@ -906,23 +965,24 @@ __global__ void zs_vote_apply_kernel(WsHeader* ws, int speculative, float max_no
 //     fp16 parameters from the unchanged live master; also zero_cast_params
 // ---------------------------------------------------------------------------
 
-template <bool VEC, bool BF>
-__device__ __forceinline__ void cast_segments(const float* master, uint16_t* params, const SegList& segs)
+template <bool VEC, bool BF, bool PEER>
+__device__ __forceinline__ void cast_segments(const float* master, uint16_t* params, const SegList& segs,
+                                              const PeerParam<PEER>& pt)
 {
     walk_segments<VEC>(
         segs,
         [&](const Seg& sg, int64_t e) {
             float p[8];
             ld_f8(master + sg.s_off + e, p);
-            __stcs(reinterpret_cast<uint4*>(params + sg.p_off + e), pack_h8<BF>(p));
+            store_params8<PEER>(params, pt, sg.p_off + e, pack_h8<BF>(p));
         },
-        [&](const Seg& sg, int64_t e) { params[sg.p_off + e] = f2h<BF>(master[sg.s_off + e]); });
+        [&](const Seg& sg, int64_t e) { store_param1<PEER>(params, pt, sg.p_off + e, f2h<BF>(master[sg.s_off + e])); });
 }
 
-template <bool VEC, bool BF>
+template <bool VEC, bool BF, bool PEER>
 __global__ void __launch_bounds__(kThreads)
 zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int bookkeeping,
-                 zero_opt_state* st, zero_step_result* res)
+                 zero_opt_state* st, zero_step_result* res, const __grid_constant__ PeerParam<PEER> pt)
 {
     wait_for_predecessor();
     const WsHeader* ws = a.ws;
@@ -952,14 +1012,14 @@ zs_commit_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int b
     }
     if (!over)
         return;
-    cast_segments<VEC, BF>(cur ? a.master[1] : a.master[0], a.params, segs);
+    cast_segments<VEC, BF, PEER>(cur ? a.master[1] : a.master[0], a.params, segs, pt);
 }
 
 template <bool VEC, bool BF>
 __global__ void __launch_bounds__(kThreads)
 zs_cast_kernel(const float* master, uint16_t* params, const __grid_constant__ SegList segs)
 {
-    cast_segments<VEC, BF>(master, params, segs);
+    cast_segments<VEC, BF, false>(master, params, segs, NoPeers{});
 }
 
 // ---------------------------------------------------------------------------
@@ -1114,24 +1174,46 @@ cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, flo
     return cudaGetLastError();
 }
 
-template <int SRC, bool VEC, bool BF>
-static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+// The peer table as the kernel parameter of a PEER / non-PEER instantiation.
+template <bool PEER>
+static PeerParam<PEER> peer_param(const PeerTable* peers)
 {
+    if constexpr (PEER)
+        return *peers;
+    else
+        return NoPeers{};
+}
+
+template <int SRC, bool VEC, bool BF, bool PEER>
+static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, const PeerTable* peers, cudaStream_t s)
+{
+    auto kernel = zs_update_kernel<SRC, VEC, BF, PEER>;
     int blocks = 0;
-    cudaError_t e = grid_for(zs_update_kernel<SRC, VEC, BF>, seg_work(segs, VEC), 0, &blocks);
+    cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = launch_overlapped(zs_update_kernel<SRC, VEC, BF>, blocks, kThreads, 0, s, a, segs);
+    e = launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, peer_param<PEER>(peers));
     count_launches(1);
     return e;
 }
 
-template <int SRC>
-static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+template <int SRC, bool BF>
+static cudaError_t launch_update_v(bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
+                                   cudaStream_t s)
 {
-    if (a.bf16)
-        return vec ? launch_update_t<SRC, true, true>(a, segs, s) : launch_update_t<SRC, false, true>(a, segs, s);
-    return vec ? launch_update_t<SRC, true, false>(a, segs, s) : launch_update_t<SRC, false, false>(a, segs, s);
+    if (peers)
+        return vec ? launch_update_t<SRC, true, BF, true>(a, segs, peers, s)
+                   : launch_update_t<SRC, false, BF, true>(a, segs, peers, s);
+    return vec ? launch_update_t<SRC, true, BF, false>(a, segs, peers, s)
+               : launch_update_t<SRC, false, BF, false>(a, segs, peers, s);
+}
+
+template <int SRC>
+static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
+                                      cudaStream_t s)
+{
+    return a.bf16 ? launch_update_v<SRC, true>(vec, a, segs, peers, s)
+                  : launch_update_v<SRC, false>(vec, a, segs, peers, s);
 }
 
 // Shape of the pipelined update for a given source: elements per consumer
@@ -1168,10 +1250,11 @@ static bool pipe_shape(int src, int nd, PipeShape* ps)
 
 static std::map<std::pair<const void*, int>, int> g_smem_set; // (kernel, device) -> bytes allowed
 
-template <int SRC, int EPT, bool BF>
-static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+template <int SRC, int EPT, bool BF, bool PEER>
+static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
+                                 const PeerTable* peers, cudaStream_t s)
 {
-    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF>;
+    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER>;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || (e = device_sms(&sms)) != cudaSuccess)
@@ -1194,26 +1277,37 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
     int64_t grid = (int64_t)sms * ps.ctas_per_sm;
     grid = tiles < grid ? tiles : grid;
     grid = grid < 1 ? 1 : grid;
-    e = launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages);
+    e = launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages,
+                          peer_param<PEER>(peers));
     count_launches(1);
     return e;
 }
 
-template <int SRC, bool BF>
-static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+template <int SRC, bool BF, bool PEER>
+static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
+                                 const PeerTable* peers, cudaStream_t s)
 {
     switch (ps.ept) {
-    case 8: return launch_pipe_t<SRC, 8, BF>(a, segs, ps, s);
-    case 4: return launch_pipe_t<SRC, 4, BF>(a, segs, ps, s);
-    case 2: return launch_pipe_t<SRC, 2, BF>(a, segs, ps, s);
-    default: return launch_pipe_t<SRC, 1, BF>(a, segs, ps, s);
+    case 8: return launch_pipe_t<SRC, 8, BF, PEER>(a, segs, ps, peers, s);
+    case 4: return launch_pipe_t<SRC, 4, BF, PEER>(a, segs, ps, peers, s);
+    case 2: return launch_pipe_t<SRC, 2, BF, PEER>(a, segs, ps, peers, s);
+    default: return launch_pipe_t<SRC, 1, BF, PEER>(a, segs, ps, peers, s);
     }
 }
 
+// With peer tables the pipeline runs only from the stash (its rank loads stay
+// on the register path); the stash pipeline then stores to every destination.
 template <int SRC>
-static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const PipeShape& ps, cudaStream_t s)
+static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
+                               const PeerTable* peers, cudaStream_t s)
 {
-    return a.bf16 ? launch_pipe_f<SRC, true>(a, segs, ps, s) : launch_pipe_f<SRC, false>(a, segs, ps, s);
+    if constexpr (SRC == kSrcStash) {
+        if (peers)
+            return a.bf16 ? launch_pipe_f<SRC, true, true>(a, segs, ps, peers, s)
+                          : launch_pipe_f<SRC, false, true>(a, segs, ps, peers, s);
+    }
+    return a.bf16 ? launch_pipe_f<SRC, true, false>(a, segs, ps, nullptr, s)
+                  : launch_pipe_f<SRC, false, false>(a, segs, ps, nullptr, s);
 }
 
 // The bulk-copy pipeline pays off where a parameter carries few bytes (the
@@ -1223,20 +1317,21 @@ static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const P
 // (0.95-1.02 against 0.64-0.95).
 static bool use_pipeline(int src, int nd) { return src == kSrcStash || nd <= 2; }
 
-cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, cudaStream_t s)
+cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
+                          cudaStream_t s)
 {
     PipeShape ps;
-    if (vec && use_pipeline(src, a.nd) && pipe_shape(src, a.nd, &ps)) {
+    if (vec && use_pipeline(src, a.nd) && (!peers || src == kSrcStash) && pipe_shape(src, a.nd, &ps)) {
         switch (src) {
-        case kSrcGradsSpeculative: return launch_pipe<kSrcGradsSpeculative>(a, segs, ps, s);
-        case kSrcGradsInPlace: return launch_pipe<kSrcGradsInPlace>(a, segs, ps, s);
-        default: return launch_pipe<kSrcStash>(a, segs, ps, s);
+        case kSrcGradsSpeculative: return launch_pipe<kSrcGradsSpeculative>(a, segs, ps, nullptr, s);
+        case kSrcGradsInPlace: return launch_pipe<kSrcGradsInPlace>(a, segs, ps, nullptr, s);
+        default: return launch_pipe<kSrcStash>(a, segs, ps, peers, s);
         }
     }
     switch (src) {
-    case kSrcGradsSpeculative: return launch_update_regs<kSrcGradsSpeculative>(vec, a, segs, s);
-    case kSrcGradsInPlace: return launch_update_regs<kSrcGradsInPlace>(vec, a, segs, s);
-    default: return launch_update_regs<kSrcStash>(vec, a, segs, s);
+    case kSrcGradsSpeculative: return launch_update_regs<kSrcGradsSpeculative>(vec, a, segs, peers, s);
+    case kSrcGradsInPlace: return launch_update_regs<kSrcGradsInPlace>(vec, a, segs, peers, s);
+    default: return launch_update_regs<kSrcStash>(vec, a, segs, peers, s);
     }
 }
 
@@ -1248,27 +1343,34 @@ int stats_blocks(bool vec, const SegList& segs)
     return (int)(want < 1 ? 1 : (want > kStatsMaxBlocks ? kStatsMaxBlocks : want));
 }
 
-template <bool VEC, bool STASH, bool BF>
-static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, cudaStream_t s)
+template <bool VEC, bool STASH, bool BF, bool PEER>
+static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, const PeerTable* peers, cudaStream_t s)
 {
-    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH, BF>, stats_blocks(VEC, segs), kThreads,
-                                            0, s, a, segs);
+    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH, BF, PEER>, stats_blocks(VEC, segs),
+                                            kThreads, 0, s, a, segs, peer_param<PEER>(peers));
     count_launches(1);
     return e;
 }
 
-template <bool BF>
-static cudaError_t launch_stats_f(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
+template <bool BF, bool PEER>
+static cudaError_t launch_stats_f(bool vec, const StatsArgs& a, const SegList& segs, const PeerTable* peers,
+                                  cudaStream_t s)
 {
     const bool stash = a.stash != nullptr;
     if (vec)
-        return stash ? launch_stats_t<true, true, BF>(a, segs, s) : launch_stats_t<true, false, BF>(a, segs, s);
-    return stash ? launch_stats_t<false, true, BF>(a, segs, s) : launch_stats_t<false, false, BF>(a, segs, s);
+        return stash ? launch_stats_t<true, true, BF, PEER>(a, segs, peers, s)
+                     : launch_stats_t<true, false, BF, PEER>(a, segs, peers, s);
+    return stash ? launch_stats_t<false, true, BF, PEER>(a, segs, peers, s)
+                 : launch_stats_t<false, false, BF, PEER>(a, segs, peers, s);
 }
 
-cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s)
+cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, const PeerTable* peers, cudaStream_t s)
 {
-    return a.bf16 ? launch_stats_f<true>(vec, a, segs, s) : launch_stats_f<false>(vec, a, segs, s);
+    if (peers)
+        return a.bf16 ? launch_stats_f<true, true>(vec, a, segs, peers, s)
+                      : launch_stats_f<false, true>(vec, a, segs, peers, s);
+    return a.bf16 ? launch_stats_f<true, false>(vec, a, segs, peers, s)
+                  : launch_stats_f<false, false>(vec, a, segs, peers, s);
 }
 
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, float max_norm,
@@ -1296,27 +1398,37 @@ cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, ze
     return cudaGetLastError();
 }
 
-template <bool VEC, bool BF>
+template <bool VEC, bool BF, bool PEER>
 static cudaError_t launch_commit_t(const UpdateArgs& a, const SegList& segs, bool bookkeeping, zero_opt_state* st,
-                                   zero_step_result* res, cudaStream_t s)
+                                   zero_step_result* res, const PeerTable* peers, cudaStream_t s)
 {
+    auto kernel = zs_commit_kernel<VEC, BF, PEER>;
     int blocks = 0;
-    cudaError_t e = grid_for(zs_commit_kernel<VEC, BF>, seg_work(segs, VEC), 0, &blocks);
+    cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = launch_overlapped(zs_commit_kernel<VEC, BF>, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res);
+    e = launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res,
+                          peer_param<PEER>(peers));
     count_launches(1);
     return e;
 }
 
-cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
-                          zero_opt_state* st, zero_step_result* res, cudaStream_t s)
+template <bool BF, bool PEER>
+static cudaError_t launch_commit_f(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
+                                   zero_opt_state* st, zero_step_result* res, const PeerTable* peers, cudaStream_t s)
 {
-    if (a.bf16)
-        return vec ? launch_commit_t<true, true>(a, segs, bookkeeping, st, res, s)
-                   : launch_commit_t<false, true>(a, segs, bookkeeping, st, res, s);
-    return vec ? launch_commit_t<true, false>(a, segs, bookkeeping, st, res, s)
-               : launch_commit_t<false, false>(a, segs, bookkeeping, st, res, s);
+    return vec ? launch_commit_t<true, BF, PEER>(a, segs, bookkeeping, st, res, peers, s)
+               : launch_commit_t<false, BF, PEER>(a, segs, bookkeeping, st, res, peers, s);
+}
+
+cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
+                          zero_opt_state* st, zero_step_result* res, const PeerTable* peers, cudaStream_t s)
+{
+    if (peers)
+        return a.bf16 ? launch_commit_f<true, true>(vec, a, segs, bookkeeping, st, res, peers, s)
+                      : launch_commit_f<false, true>(vec, a, segs, bookkeeping, st, res, peers, s);
+    return a.bf16 ? launch_commit_f<true, false>(vec, a, segs, bookkeeping, st, res, peers, s)
+                  : launch_commit_f<false, false>(vec, a, segs, bookkeeping, st, res, peers, s);
 }
 
 template <bool VEC, bool BF>

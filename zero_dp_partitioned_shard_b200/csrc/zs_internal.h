@@ -110,6 +110,17 @@ struct StatsArgs {
     int32_t bf16;             // 16-bit storage of the contributions: 0 fp16, 1 bf16
 };
 
+// Peer tables of a fused reduce-scatter + update + all-gather call (kernel
+// parameter, 1 KiB): rank r's contribution to flat element f is at
+// grads[r][f]; each new parameter is stored at params[p] and dests[d][p].
+constexpr int kMaxPeers = ZERO_MAX_PEERS;
+struct PeerTable {
+    const uint16_t* grads[kMaxPeers];
+    uint16_t* dests[kMaxPeers];
+    int32_t n_dests;
+    int32_t pad;
+};
+
 struct GatherEntry {
     const uint16_t* src;
     int64_t dst_off;
@@ -128,11 +139,13 @@ cudaError_t launch_opt_init(zero_opt_state* st, float scale, float growth, float
                             cudaStream_t s);
 cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2, float static_inv,
                         double scale_mult, cudaStream_t s);
+// peers: nullptr for the strided addressing of UpdateArgs / StatsArgs
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs,
-                          cudaStream_t s);
+                          const PeerTable* peers, cudaStream_t s);
 // blocks (= fp64 partials written) of one statistics launch over segs
 int stats_blocks(bool vec, const SegList& segs);
-cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cudaStream_t s);
+cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, const PeerTable* peers,
+                         cudaStream_t s);
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n_partials,
                             float max_grad_norm, zero_opt_state* st, zero_step_result* res,
                             cudaStream_t s);
@@ -140,7 +153,7 @@ cudaError_t launch_vote_local(WsHeader* ws, const double* partials, int64_t n, c
 cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, zero_opt_state* st,
                               zero_step_result* res, cudaStream_t s);
 cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bool bookkeeping,
-                          zero_opt_state* st, zero_step_result* res, cudaStream_t s);
+                          zero_opt_state* st, zero_step_result* res, const PeerTable* peers, cudaStream_t s);
 cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
                         cudaStream_t s);
 cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s);
