@@ -70,7 +70,7 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
 
     class Args:
-        steps, warmup, ref_sample = 1, 3, 1000
+        steps, warmup, ref_sample, storage = 1, 3, 1000, "fp16"
     wl = bench._workloads()["gpt2-1.5b-stage2-nd8"]
     assert bench.run_reference(Args, "gpt2-1.5b-stage2-nd8", wl) == 0
     assert capsys.readouterr().out == ""
