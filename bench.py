@@ -17,6 +17,11 @@ reports the update kernel's algorithmic bytes per launch over its CUDA-event
 duration against the measured HBM copy bandwidth; ``cpu_baseline`` times the
 CPU oracle on a bounded sample on this host.
 
+``--peer`` runs the same step through peer tables with the Nd ranks' buffers
+in this GPU's memory: each rank's gradient read through the table, every new
+parameter stored into all Nd full parameter buffers (the all-gather by
+stores), which adds 2 (Nd - 1) bytes per parameter.
+
 Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): the path has
 no data exchange on one GPU, so N ranks run independent replicas (weak
 scaling); the only collectives are the timing barrier and the max over ranks.
@@ -75,11 +80,12 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     return alg, moved
 
 
-def update_launch_bytes(nd: int, mode: int) -> int:
+def update_launch_bytes(nd: int, mode: int, dests: int = 0) -> int:
     """Algorithmic bytes per parameter of the update kernel's own launch: the
     fused kernel reads the Nd contributions (speculative, two-pass) or the
-    4-byte stash (stash), plus master/m/v read and write and the fp16 write."""
-    return (4 if mode == 2 else 2 * nd) + 26
+    4-byte stash (stash), plus master/m/v read and write and the fp16 write
+    (to the parameter buffer and to each of `dests` more)."""
+    return (4 if mode == 2 else 2 * nd) + 26 + 2 * dests
 
 
 def profiled_traffic(nd: int, mode: int, owned: int):
@@ -168,7 +174,7 @@ class ClockSampler:
 class Bench:
     """Device buffers and the C-ABI arguments of one workload on one GPU."""
 
-    def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0):
+    def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0, peer: bool = False):
         import torch
         from zero_dp_partitioned_shard_b200 import binding as B
         from zero_dp_partitioned_shard_b200 import synth
@@ -241,6 +247,15 @@ class Bench:
             for k, r in enumerate(others):
                 self.shard_ptrs[r] = self.shards[k].data_ptr()
             self.assembled = sum(max(0, min(L, psi - r * L)) for r in others)
+        # peer tables: rank r's gradient is row r, every rank has its own full
+        # parameter buffer (the call's params plus Nd - 1 destinations)
+        self.dests = []
+        if peer:
+            if wl["layout"] != B.ZERO_GRADS_FULL:
+                raise ValueError("--peer needs a workload with full per-rank gradients")
+            self.dests = [torch.zeros(psi, dtype=h16, device=dev) for _ in range(self.nd - 1)]
+            rank_grads = [self.grads.data_ptr() + 2 * r * stride for r in range(self.nd)]
+            B.attach_peers(self.args, B.peer_args(rank_grads, [t.data_ptr() for t in self.dests]))
         ws_bytes = B.zero_workspace_bytes(self.plan, self.hp, self.args)
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.args.workspace = self.workspace.data_ptr()
@@ -461,6 +476,8 @@ def main():
     ap.add_argument("--psi", type=int, default=0, help="smaller Psi of the same workload (profiling)")
     ap.add_argument("--storage", choices=sorted(STORAGES), default="fp16",
                     help="16-bit format of gradients and parameters")
+    ap.add_argument("--peer", action="store_true",
+                    help="through peer tables, storing the parameters into all Nd ranks' buffers")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -488,7 +505,8 @@ def main():
     import torch
     from zero_dp_partitioned_shard_b200 import binding as B
     world, rank, local = _dist()
-    bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage])
+    bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage], peer=args.peer)
+    n_dests = len(bench.dests)
     alg, moved = bytes_per_param(wl["nd"], wl["mode"])
 
     # --- device-resident timing ---
@@ -553,20 +571,21 @@ def main():
             e2e = {"value": None, "unit": UNIT, "skipped": "host memory below 2.5x the gradient bytes"}
 
     peak, peak_kind = measured_hbm_peak()
-    k_bytes = bench.owned * update_launch_bytes(wl["nd"], wl["mode"])
+    k_bytes = bench.owned * update_launch_bytes(wl["nd"], wl["mode"], n_dests)
     achieved = k_bytes / (k_ms_max / 1e3) / 1e9
-    traffic, traffic_src = profiled_traffic(wl["nd"], wl["mode"], bench.owned)
+    traffic, traffic_src = profiled_traffic(wl["nd"], wl["mode"], bench.owned) if not n_dests else (None, None)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": args.workload, "description": wl["desc"], "psi": bench.psi,
                    "nd": wl["nd"], "stage": wl["stage"], "storage": args.storage,
+                   "peer_tables": bool(n_dests), "param_dests": n_dests,
                    "owned_params_per_gpu": bench.owned,
                    "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
                    "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
                    "assembled_params": bench.assembled,
-                   "step_gbs_alg": (bench.owned * alg + 4 * bench.assembled)
+                   "step_gbs_alg": (bench.owned * (alg + 2 * n_dests) + 4 * bench.assembled)
                                    / (ms_max / args.steps / 1e3) / 1e9,
                    "l2": "inputs larger than L2 (no flush): "
                          f"{bench.owned * moved / 1e9:.1f} GB moved per step",
