@@ -89,6 +89,7 @@ def lib():
             "oracle_state_bytes": (C.c_int, [_I64, _I32, _I32, _I64, C.POINTER(StateReport)]),
             "oracle_all_reduce": (None, [_P, _I64, _I32, _I64, _P]),
             "oracle_reduce_scatter": (None, [_P, _I64, C.POINTER(PlanT), _P]),
+            "oracle_reduce_scatter16": (None, [_P, _I64, C.POINTER(PlanT), _I32, _I64, _I64, _P]),
             "oracle_all_gather_f32": (None, [_P, C.POINTER(PlanT), _P]),
             "oracle_gather_params": (None, [_P, C.POINTER(PlanT), _P]),
             "oracle_gather_tensors": (_I64, [C.POINTER(PlanT), _P, _I32, _I32, _I32, _P, _P, _I32]),
@@ -223,6 +224,23 @@ def reduce_scatter(G: np.ndarray, p: Plan) -> np.ndarray:
     out = np.empty((p.nd, p.shard_len), dtype=np.float32)
     pc = p._c()
     lib().oracle_reduce_scatter(_ptr(G), G.shape[1], C.byref(pc), _ptr(out))
+    return out
+
+
+def reduce_scatter16(G: np.ndarray, p: Plan, storage: int = 0, lo: int = 0, hi: int | None = None,
+                     out: np.ndarray | None = None) -> np.ndarray:
+    """The owners' retained 16-bit reduced gradients [nd, L] (uint16 bits):
+    the rank-order fp32 sum rounded once to the storage format, written for
+    flat indices in [lo, hi) only (into ``out`` if given; fresh pads are
+    0xFFFF, a NaN in both formats, and are never written)."""
+    G = np.ascontiguousarray(G, dtype=np.uint16)
+    assert G.shape[0] == p.nd and G.shape[1] >= p.psi
+    hi = p.psi if hi is None else hi
+    if out is None:
+        out = np.full((p.nd, p.shard_len), 0xFFFF, dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.flags.c_contiguous and out.size == p.nd * p.shard_len
+    pc = p._c()
+    lib().oracle_reduce_scatter16(_ptr(G), G.shape[1], C.byref(pc), int(storage), int(lo), int(hi), _ptr(out))
     return out
 
 

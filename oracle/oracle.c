@@ -46,6 +46,9 @@
  *   - Bias corrections: running products beta^t in fp64, 1 - beta^t rounded
  *     to fp32.
  *   - Padding: equal shards of L = ceil(Psi/(Nd*A))*A elements.
+ *   - Stage-2 retention: the gradient an owner keeps after the reduce-scatter
+ *     is that fp32 sum rounded once (to nearest even) to the gradients'
+ *     16-bit format.
  *
  * Every function here is pinned by a CPU test against values the pages print,
  * closed forms or library routines (tests/test_oracle_*.py).  Nothing is
@@ -395,6 +398,28 @@ void oracle_reduce_scatter(const uint16_t* G, int64_t rank_stride, const oracle_
         float* dst = shards + (int64_t)o * p->shard_len;
         for (int64_t i = 0; i < p->shard_len; ++i)
             dst[i] = i < len ? rank_sum(G, rank_stride, p->nd, start + i) : 0.0f;
+    }
+}
+
+/* Reduce-scatter with retention (stage 2, P_os+g): each gradient element is
+ * reduced only on the process that owns its partition, which keeps it, and
+ * the ranks' full gradients are released ([Guide] "How it works"; [Dissect]
+ * "ZeRO-2: Also Partition the Gradients").  What is kept is the reduced
+ * gradient in the gradients' own 16-bit format (storage 0: fp16, 1: bf16):
+ * the rank-order fp32 sum, rounded once.  shards is [Nd][L]; only the flat
+ * range [lo, hi) is written (one bucket, or everything), pads never. */
+void oracle_reduce_scatter16(const uint16_t* G, int64_t rank_stride, const oracle_plan_t* p, int32_t storage,
+                             int64_t lo, int64_t hi, uint16_t* shards)
+{
+    for (int32_t o = 0; o < p->nd; ++o) {
+        int64_t start, len;
+        oracle_shard(p, o, &start, &len);
+        uint16_t* dst = shards + (int64_t)o * p->shard_len;
+        for (int64_t i = 0; i < len; ++i) {
+            const int64_t f = start + i;
+            if (f >= lo && f < hi)
+                dst[i] = to_storage(rank_sum_of(G, rank_stride, p->nd, f, storage), storage);
+        }
     }
 }
 
