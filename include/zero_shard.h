@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 5
+#define ZERO_SHARD_ABI_VERSION 6
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -107,9 +107,15 @@ typedef int32_t zero_status;
  *   PER_OWNER (stage 3: contributions arrive already partitioned): rank r's
  *     contribution to element i of owner (owner_first + k) is
  *     grads[(k * nd + r) * grad_rank_stride + i], grad_rank_stride >= L
- *     (0 means L). */
+ *     (0 means L).
+ *   REDUCED (stage 2 with retention): the owners' reduced gradients as
+ *     zero_reduce_scatter keeps them, one value per element: element i of
+ *     owner (owner_first + k) is grads[k * L + i]; grad_rank_stride is
+ *     ignored.  The step then sums nothing and otherwise runs unchanged
+ *     (averaging still divides by the plan's nd). */
 #define ZERO_GRADS_FULL 0
 #define ZERO_GRADS_PER_OWNER 1
+#define ZERO_GRADS_REDUCED 2
 
 /* 16-bit format of the gradient contributions and of the parameters.  The
  * pages' mixed precision uses fp16; bfloat16 (the same 2 bytes, the upper half
@@ -303,7 +309,7 @@ typedef struct zero_step_args {
  *   Entries past nd / n_param_dests are ignored.  The arithmetic and the
  *   results are exactly those of the strided call with the same data.
  * Errors (besides zero_shard_step's): UNSUPPORTED if nd > ZERO_MAX_PEERS or
- * grad_layout is PER_OWNER; INVALID_ARG for a NULL entry or n_param_dests
+ * grad_layout is not FULL; INVALID_ARG for a NULL entry or n_param_dests
  * outside [0, ZERO_MAX_PEERS]; ALIGNMENT for an entry not 2-byte aligned
  * (16-byte aligned entries keep the vectorised path). */
 #define ZERO_MAX_PEERS 64
@@ -428,6 +434,32 @@ ZERO_API zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hpa
  *     norm: order them, e.g. on one stream. */
 ZERO_API zero_status zero_shard_step_static_scratch(const zero_plan_t* plan, const zero_hparams* hp,
                                                     const zero_step_args* args, void* stream);
+
+/* Reduce-scatter with retention (ZeRO stage 2, P_os+g): each gradient is
+ * reduced only on the process that owns its partition, which keeps the
+ * result, and the full gradients can then be released -- "ZeRO: partitioning
+ * training state across GPUs" (upskillscore.com), "How it works";
+ * "ZeRO memory optimization" (trishampatil.com), "ZeRO-2".
+ *   For the owners owner_first .. owner_first + owner_count - 1 of args and
+ *   the flat range of bucket `bucket` of the plan (bucket < 0: the owners'
+ *   whole range; a plan without buckets has the one bucket 0), writes
+ *   grad_shards[k * L + i] = the rank-order fp32 sum of the Nd
+ *   contributions to element i of owner (owner_first + k), rounded once to
+ *   nearest even in args->storage's 16-bit format.  Pads (i >= real_len)
+ *   and elements outside the bucket are not written.
+ *   The contributions come from args->grads in args->grad_layout (FULL or
+ *   PER_OWNER) or through args->peers; every other field of args is
+ *   ignored.  grad_shards: device, owner_count * L 16-bit values; a
+ *   16-byte aligned buffer (with 16-byte aligned contributions) takes the
+ *   vectorised path.
+ *   The step consumes the result with grad_layout = ZERO_GRADS_REDUCED.  A
+ *   sum beyond the format's range is kept as inf and skips that step.
+ *   Bucket by bucket, a caller can reduce each bucket as soon as every rank
+ *   has produced it and then reuse the ranks' buffers for it.
+ * Errors: INVALID_ARG (null pointers, owner range, layout, bucket outside
+ * [0, n_buckets)), ALIGNMENT, UNSUPPORTED (peer-table limits), CUDA. */
+ZERO_API zero_status zero_reduce_scatter(const zero_plan_t* plan, const zero_step_args* args, int64_t bucket,
+                                         void* grad_shards, void* stream);
 
 /* Gather-assembly (the stage-3 all-gather seen by one rank): for every owner
  * r whose shard_ptrs[r] (host array of nd device pointers) is not NULL,

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
     lib = B.lib()
     for name in declared:
         assert getattr(lib, name) is not None
-    assert B.zero_abi_version() == 5
+    assert B.zero_abi_version() == 6
     # nothing else leaks out of the library (hidden visibility)
     assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
 
@@ -278,6 +278,39 @@ def test_peer_tables_replace_the_strided_gradients():
         assert e.value.status == B.ZERO_ERR_UNSUPPORTED
     finally:
         B.zero_plan_destroy(big)
+
+
+def test_reduced_layout_and_reduce_scatter_validation():
+    """The REDUCED layout takes one value per element (no stride); the
+    reduce-scatter with retention accepts FULL / PER_OWNER sources only, a
+    bucket inside the plan and a 2-byte aligned destination."""
+    plan = B.zero_plan(1000, 4, stage=2, align_elems=8, bucket_elems=300)
+    hp = B.hparams(loss_scale=1.0)
+    lib = B.lib()
+    try:
+        red = _args(grad_layout=B.ZERO_GRADS_REDUCED, grad_rank_stride=0)
+        assert B.zero_workspace_bytes(plan, hp, red) == 256
+        q = B.peer_args([FAKE] * 4)
+        with pytest.raises(B.ZeroError) as e:
+            B.zero_workspace_bytes(plan, hp, B.attach_peers(_args(grad_layout=B.ZERO_GRADS_REDUCED), q))
+        assert e.value.status == B.ZERO_ERR_UNSUPPORTED
+
+        def reduce_status(args, bucket, out):
+            before = B.zero_launch_count()
+            st = lib.zero_reduce_scatter(plan, C.byref(args), bucket, out, None)
+            assert B.zero_launch_count() == before        # rejected before any launch
+            return st
+
+        full = _args()
+        assert reduce_status(full, 4, FAKE) == B.ZERO_ERR_INVALID_ARG           # 4 buckets: 0..3
+        assert reduce_status(full, 0, None) == B.ZERO_ERR_INVALID_ARG
+        assert reduce_status(full, 0, FAKE + 1) == B.ZERO_ERR_ALIGNMENT
+        assert reduce_status(red, 0, FAKE) == B.ZERO_ERR_INVALID_ARG            # REDUCED is not a source
+        assert reduce_status(_args(grads=0), 0, FAKE) == B.ZERO_ERR_INVALID_ARG
+        assert reduce_status(_args(owner_first=3, owner_count=2), 0, FAKE) == B.ZERO_ERR_INVALID_ARG
+        assert reduce_status(_args(grad_rank_stride=999), -1, FAKE) == B.ZERO_ERR_INVALID_ARG
+    finally:
+        B.zero_plan_destroy(plan)
 
 
 def test_ipc_helpers_validate_arguments():

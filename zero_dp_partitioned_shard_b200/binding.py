@@ -32,6 +32,7 @@ ZERO_MODE_STASH = 2
 
 ZERO_GRADS_FULL = 0
 ZERO_GRADS_PER_OWNER = 1
+ZERO_GRADS_REDUCED = 2
 
 ZERO_STORAGE_FP16 = 0
 ZERO_STORAGE_BF16 = 1
@@ -141,6 +142,7 @@ SIGNATURES = {
     "zero_shard_step_begin": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_end": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
+    "zero_reduce_scatter": (_S, [_P, C.POINTER(StepArgs), C.c_int64, _P, _P]),
     "zero_gather_tensors": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, C.c_int32, _P]),
     "zero_ipc_export": (_S, [_P, C.POINTER(IpcHandle)]),
@@ -167,7 +169,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 5:
+        if L.zero_abi_version() != 6:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -270,6 +272,12 @@ def zero_shard_step_begin(plan: int, hp: HParams, args: StepArgs, stream: int = 
 def zero_shard_step_end(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
     """Second half of a split step, after the votes of all owners were summed in place."""
     _check(lib().zero_shard_step_end(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step_end")
+
+
+def zero_reduce_scatter(plan: int, args: StepArgs, grad_shards: int, bucket: int = -1, stream: int = 0) -> None:
+    """Keeps the owners' reduced gradients (16-bit, [owner_count * L]) for a
+    later step with grad_layout ZERO_GRADS_REDUCED; bucket < 0: everything."""
+    _check(lib().zero_reduce_scatter(plan, C.byref(args), bucket, grad_shards, stream), "zero_reduce_scatter")
 
 
 def zero_gather_params(plan: int, shard_ptrs, params_full: int, stream: int = 0) -> None:

@@ -37,6 +37,8 @@ void push_seg(std::vector<zs::SegList>& lists, const zs::Seg& s)
 void segments_of(const zero_plan_s& p, int layout, int64_t stride, int32_t o0, int64_t lo,
                  int64_t hi, std::vector<zs::SegList>& out)
 {
+    // per-owner blocks hold nd contributions (PER_OWNER) or one (REDUCED)
+    const int64_t per_owner = layout == ZERO_GRADS_REDUCED ? 1 : p.nd;
     const int64_t L = p.shard_len;
     if (lo >= hi)
         return;
@@ -49,7 +51,7 @@ void segments_of(const zero_plan_s& p, int layout, int64_t stride, int32_t o0, i
         const int64_t i0 = (lo > o * L ? lo : o * L) - o * L;
         const int64_t i1 = (hi < (o + 1) * L ? hi : (o + 1) * L) - o * L;
         const int64_t j = o - o0;
-        push_seg(out, zs::Seg{j * p.nd * stride + i0, stride, j * L + i0, o * L + i0, i1 - i0});
+        push_seg(out, zs::Seg{j * per_owner * stride + i0, stride, j * L + i0, o * L + i0, i1 - i0});
     }
 }
 
@@ -66,38 +68,26 @@ int64_t effective_stride(const zero_plan_s& p, const zero_step_args& a)
 {
     if (a.peers) // one buffer per rank: the stride is not used
         return 0;
+    if (a.grad_layout == ZERO_GRADS_REDUCED) // one value per element, owners back to back
+        return p.shard_len;
     if (a.grad_layout == ZERO_GRADS_PER_OWNER && a.grad_rank_stride == 0)
         return p.shard_len;
     return a.grad_rank_stride;
 }
 
-zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_step_args* a)
+// Checks of where a call's gradient contributions come from and which owners
+// it covers (zero_shard_step and zero_reduce_scatter).  reduced_ok: the
+// REDUCED layout is accepted (the step's input, not the reduce-scatter's).
+zero_status validate_source(const zero_plan_s* p, const zero_step_args* a, bool reduced_ok)
 {
-    if (!p || !hp || !a)
-        return fail(ZERO_ERR_INVALID_ARG, "zero_shard_step: null plan, hparams or args");
-    if (hp->mode < ZERO_MODE_SPECULATIVE || hp->mode > ZERO_MODE_STASH)
-        return fail(ZERO_ERR_INVALID_ARG, "unknown mode %d", hp->mode);
-    if (hp->reserved != 0)
-        return fail(ZERO_ERR_INVALID_ARG, "reserved fields must be 0");
     if (a->storage != ZERO_STORAGE_FP16 && a->storage != ZERO_STORAGE_BF16)
         return fail(ZERO_ERR_INVALID_ARG, "unknown 16-bit storage format %d", a->storage);
-    if (!(hp->loss_scale > 0.0f) || !std::isfinite(hp->loss_scale))
-        return fail(ZERO_ERR_INVALID_ARG, "loss_scale must be finite and > 0");
-    if (!std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay) || !std::isfinite(hp->eps) ||
-        hp->eps < 0.0f || !std::isfinite(hp->max_grad_norm))
-        return fail(ZERO_ERR_INVALID_ARG, "lr, weight_decay, eps, max_grad_norm must be finite, eps >= 0");
-    if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f))
-        return fail(ZERO_ERR_INVALID_ARG, "betas must lie in [0, 1)");
-    if (hp->average_over_nd != 0 && hp->average_over_nd != 1)
-        return fail(ZERO_ERR_INVALID_ARG, "average_over_nd must be 0 or 1");
-    if (hp->mode == ZERO_MODE_SPECULATIVE && hp->max_grad_norm > 0.0f)
-        return fail(ZERO_ERR_UNSUPPORTED, "global-norm clipping needs the norm before any update: "
-                    "use TWO_PASS or STASH mode");
     if (a->owner_first < 0 || a->owner_count < 1 || a->owner_first > p->nd - a->owner_count)
         return fail(ZERO_ERR_INVALID_ARG, "owner range [%d, %d + %d) outside [0, %d)",
                     a->owner_first, a->owner_first, a->owner_count, p->nd);
-    if (a->grad_layout != ZERO_GRADS_FULL && a->grad_layout != ZERO_GRADS_PER_OWNER)
-        return fail(ZERO_ERR_INVALID_ARG, "unknown grad_layout %d", a->grad_layout);
+    const bool reduced = a->grad_layout == ZERO_GRADS_REDUCED;
+    if (a->grad_layout != ZERO_GRADS_FULL && a->grad_layout != ZERO_GRADS_PER_OWNER && !(reduced && reduced_ok))
+        return fail(ZERO_ERR_INVALID_ARG, "grad_layout %d not accepted here", a->grad_layout);
     if (a->peers) {
         const zero_peer_args& q = *a->peers;
         if (a->grad_layout != ZERO_GRADS_FULL)
@@ -120,17 +110,47 @@ zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_st
             if (!aligned(q.param_dests[d], 2))
                 return fail(ZERO_ERR_ALIGNMENT, "param_dests[%d] must be 2-byte aligned", d);
         }
+        return ZERO_OK;
     }
     const int64_t stride = effective_stride(*p, *a);
-    if (!a->peers && a->grad_layout == ZERO_GRADS_FULL && p->nd > 1 && stride < p->psi)
+    if (a->grad_layout == ZERO_GRADS_FULL && p->nd > 1 && stride < p->psi)
         return fail(ZERO_ERR_INVALID_ARG, "FULL layout needs grad_rank_stride >= psi (%lld < %lld)",
                     (long long)stride, (long long)p->psi);
     if (a->grad_layout == ZERO_GRADS_PER_OWNER && stride < p->shard_len)
         return fail(ZERO_ERR_INVALID_ARG, "PER_OWNER layout needs grad_rank_stride >= L (%lld < %lld)",
                     (long long)stride, (long long)p->shard_len);
-    if ((!a->grads && !a->peers) || !a->master[0] || !a->exp_avg[0] || !a->exp_avg_sq[0] || !a->params ||
-        !a->opt_state)
-        return fail(ZERO_ERR_INVALID_ARG, "null device buffer (grads, master, exp_avg, exp_avg_sq, params, opt_state)");
+    if (!a->grads)
+        return fail(ZERO_ERR_INVALID_ARG, "null grads");
+    if (!aligned(a->grads, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "16-bit buffers must be 2-byte aligned");
+    return ZERO_OK;
+}
+
+zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_step_args* a)
+{
+    if (!p || !hp || !a)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_shard_step: null plan, hparams or args");
+    if (hp->mode < ZERO_MODE_SPECULATIVE || hp->mode > ZERO_MODE_STASH)
+        return fail(ZERO_ERR_INVALID_ARG, "unknown mode %d", hp->mode);
+    if (hp->reserved != 0)
+        return fail(ZERO_ERR_INVALID_ARG, "reserved fields must be 0");
+    if (!(hp->loss_scale > 0.0f) || !std::isfinite(hp->loss_scale))
+        return fail(ZERO_ERR_INVALID_ARG, "loss_scale must be finite and > 0");
+    if (!std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay) || !std::isfinite(hp->eps) ||
+        hp->eps < 0.0f || !std::isfinite(hp->max_grad_norm))
+        return fail(ZERO_ERR_INVALID_ARG, "lr, weight_decay, eps, max_grad_norm must be finite, eps >= 0");
+    if (!(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f))
+        return fail(ZERO_ERR_INVALID_ARG, "betas must lie in [0, 1)");
+    if (hp->average_over_nd != 0 && hp->average_over_nd != 1)
+        return fail(ZERO_ERR_INVALID_ARG, "average_over_nd must be 0 or 1");
+    if (hp->mode == ZERO_MODE_SPECULATIVE && hp->max_grad_norm > 0.0f)
+        return fail(ZERO_ERR_UNSUPPORTED, "global-norm clipping needs the norm before any update: "
+                    "use TWO_PASS or STASH mode");
+    zero_status s = validate_source(p, a, true);
+    if (s != ZERO_OK)
+        return s;
+    if (!a->master[0] || !a->exp_avg[0] || !a->exp_avg_sq[0] || !a->params || !a->opt_state)
+        return fail(ZERO_ERR_INVALID_ARG, "null device buffer (master, exp_avg, exp_avg_sq, params, opt_state)");
     const bool spec = hp->mode == ZERO_MODE_SPECULATIVE;
     if (spec && (!a->master[1] || !a->exp_avg[1] || !a->exp_avg_sq[1]))
         return fail(ZERO_ERR_INVALID_ARG, "SPECULATIVE mode needs the second state slot");
@@ -139,8 +159,8 @@ zero_status validate(const zero_plan_s* p, const zero_hparams* hp, const zero_st
     for (int k = 0; k < (spec ? 2 : 1); ++k)
         if (!aligned(a->master[k], 4) || !aligned(a->exp_avg[k], 4) || !aligned(a->exp_avg_sq[k], 4))
             return fail(ZERO_ERR_ALIGNMENT, "fp32 state buffers must be 4-byte aligned");
-    if (!aligned(a->grads, 2) || !aligned(a->params, 2))
-        return fail(ZERO_ERR_ALIGNMENT, "fp16 buffers must be 2-byte aligned");
+    if (!aligned(a->params, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "16-bit buffers must be 2-byte aligned");
     if (a->grad_stash && !aligned(a->grad_stash, 4))
         return fail(ZERO_ERR_ALIGNMENT, "grad_stash must be 4-byte aligned");
     if (!aligned(a->opt_state, 8) || (a->result && !aligned(a->result, 8)))
@@ -199,6 +219,20 @@ LaunchPlan plan_launches(const zero_plan_s& p, const zero_hparams& hp, const zer
         for (const auto& l : b)
             lp.n_partials += zs::stats_blocks(vec, l);
     return lp;
+}
+
+// The peer table of a call (kernel parameter), or nullptr without peer tables.
+const zs::PeerTable* make_peer_table(const zero_plan_s& p, const zero_step_args& a, zs::PeerTable* pt)
+{
+    if (!a.peers)
+        return nullptr;
+    std::memset(pt, 0, sizeof *pt);
+    for (int r = 0; r < p.nd; ++r)
+        pt->grads[r] = static_cast<const uint16_t*>(a.peers->rank_grads[r]);
+    for (int d = 0; d < a.peers->n_param_dests; ++d)
+        pt->dests[d] = static_cast<uint16_t*>(a.peers->param_dests[d]);
+    pt->n_dests = a.peers->n_param_dests;
+    return pt;
 }
 
 size_t workspace_need(const zero_hparams& hp, const LaunchPlan& lp)
@@ -304,7 +338,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
     u.result = res;
     u.wait_budget = zs::wait_budget_cycles();
     u.bf16 = a.storage == ZERO_STORAGE_BF16 ? 1 : 0;
-    u.nd = p.nd;
+    u.nd = a.grad_layout == ZERO_GRADS_REDUCED ? 1 : p.nd; // contributions per element
     double scale = (double)h.loss_scale;
     if (h.average_over_nd)
         scale *= (double)p.nd;
@@ -320,16 +354,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
 
     // peer tables: one gradient buffer per rank, extra parameter destinations
     zs::PeerTable peer_table;
-    const zs::PeerTable* peers = nullptr;
-    if (a.peers) {
-        std::memset(&peer_table, 0, sizeof peer_table);
-        for (int r = 0; r < p.nd; ++r)
-            peer_table.grads[r] = static_cast<const uint16_t*>(a.peers->rank_grads[r]);
-        for (int d = 0; d < a.peers->n_param_dests; ++d)
-            peer_table.dests[d] = static_cast<uint16_t*>(a.peers->param_dests[d]);
-        peer_table.n_dests = a.peers->n_param_dests;
-        peers = &peer_table;
-    }
+    const zs::PeerTable* peers = make_peer_table(p, a, &peer_table);
 
     const bool spec = h.mode == ZERO_MODE_SPECULATIVE;
     const bool first_half = phase != PHASE_END;
@@ -369,7 +394,7 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
         sa.grads = u.grads;
         sa.stash = h.mode == ZERO_MODE_STASH ? a.grad_stash : nullptr;
         sa.ws = ws;
-        sa.nd = p.nd;
+        sa.nd = u.nd;
         sa.inv = u.inv;
         sa.st = st;
         sa.scale_mult = scale_mult;
@@ -402,6 +427,54 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
                 return cuda_fail(e, "update launch");
         if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
             return cuda_fail(e, "timing event");
+    }
+    return ZERO_OK;
+}
+
+zero_status zero_reduce_scatter(const zero_plan_t* plan, const zero_step_args* args, int64_t bucket,
+                                void* grad_shards, void* stream)
+{
+    zs::clear_error();
+    if (!plan || !args || !grad_shards)
+        return fail(ZERO_ERR_INVALID_ARG, "zero_reduce_scatter: null plan, args or grad_shards");
+    const zero_plan_s& p = *plan;
+    const zero_step_args& a = *args;
+    zero_status s = validate_source(&p, &a, false);
+    if (s != ZERO_OK)
+        return s;
+    if (!aligned(grad_shards, 2))
+        return fail(ZERO_ERR_ALIGNMENT, "grad_shards must be 2-byte aligned");
+    const int64_t nb = p.bucket > 0 ? p.n_buckets : 1;
+    if (bucket >= nb)
+        return fail(ZERO_ERR_INVALID_ARG, "bucket %lld outside [0, %lld)", (long long)bucket, (long long)nb);
+    const int64_t L = p.shard_len;
+    int64_t lo = (int64_t)a.owner_first * L;
+    int64_t hi = (int64_t)(a.owner_first + a.owner_count) * L;
+    hi = hi < p.psi ? hi : p.psi;
+    if (bucket >= 0 && p.bucket > 0) {
+        lo = lo > bucket * p.bucket ? lo : bucket * p.bucket;
+        hi = hi < (bucket + 1) * p.bucket ? hi : (bucket + 1) * p.bucket;
+    }
+    if (lo >= hi)
+        return ZERO_OK;
+    const int64_t stride = effective_stride(p, a);
+    std::vector<zs::SegList> lists;
+    segments_of(p, a.grad_layout, stride, a.owner_first, lo, hi, lists);
+    bool vec = (L % 8 == 0) && (stride % 8 == 0) && aligned(grad_shards, 16) && segs_vec_ok(lists);
+    if (a.peers) {
+        for (int r = 0; r < p.nd; ++r)
+            vec = vec && aligned(a.peers->rank_grads[r], 16);
+    } else {
+        vec = vec && aligned(a.grads, 16);
+    }
+    zs::PeerTable peer_table;
+    const zs::PeerTable* peers = make_peer_table(p, a, &peer_table);
+    for (const auto& l : lists) {
+        cudaError_t e = zs::launch_reduce(vec, a.storage == ZERO_STORAGE_BF16, static_cast<const uint16_t*>(a.grads),
+                                          static_cast<uint16_t*>(grad_shards), p.nd, l, peers,
+                                          static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "reduce launch");
     }
     return ZERO_OK;
 }

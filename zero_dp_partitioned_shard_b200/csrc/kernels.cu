@@ -1023,6 +1023,29 @@ zs_cast_kernel(const float* master, uint16_t* params, const __grid_constant__ Se
 }
 
 // ---------------------------------------------------------------------------
+// Reduce-scatter with retention (stage 2): the owners' reduced gradients,
+// the rank-order fp32 sum rounded once to the 16-bit format, kept at the
+// state offsets for a later step to read as its single contribution
+// ---------------------------------------------------------------------------
+
+template <bool VEC, bool BF, bool PEER>
+__global__ void __launch_bounds__(kThreads, 2)
+zs_reduce_kernel(const uint16_t* grads, uint16_t* out, int nd, const __grid_constant__ SegList segs,
+                 const __grid_constant__ PeerParam<PEER> pt)
+{
+    walk_segments<VEC>(
+        segs,
+        [&](const Seg& sg, int64_t e) {
+            float sum[8];
+            rank_sum8<BF>(ranks_at<PEER>(grads, pt, sg, e), nd, sum);
+            __stcs(reinterpret_cast<uint4*>(out + sg.s_off + e), pack_h8<BF>(sum));
+        },
+        [&](const Seg& sg, int64_t e) {
+            out[sg.s_off + e] = f2h<BF>(rank_sum1<BF>(ranks_at<PEER>(grads, pt, sg, e), nd));
+        });
+}
+
+// ---------------------------------------------------------------------------
 // K4: gather-assembly of fp16 parameter shards into the full buffer
 // ---------------------------------------------------------------------------
 
@@ -1429,6 +1452,38 @@ cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bo
                       : launch_commit_f<false, true>(vec, a, segs, bookkeeping, st, res, peers, s);
     return a.bf16 ? launch_commit_f<true, false>(vec, a, segs, bookkeeping, st, res, peers, s)
                   : launch_commit_f<false, false>(vec, a, segs, bookkeeping, st, res, peers, s);
+}
+
+template <bool VEC, bool BF, bool PEER>
+static cudaError_t launch_reduce_t(const uint16_t* grads, uint16_t* out, int nd, const SegList& segs,
+                                   const PeerTable* peers, cudaStream_t s)
+{
+    auto kernel = zs_reduce_kernel<VEC, BF, PEER>;
+    int blocks = 0;
+    cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
+    if (e != cudaSuccess)
+        return e;
+    kernel<<<blocks, kThreads, 0, s>>>(grads, out, nd, segs, peer_param<PEER>(peers));
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <bool BF, bool PEER>
+static cudaError_t launch_reduce_f(bool vec, const uint16_t* grads, uint16_t* out, int nd, const SegList& segs,
+                                   const PeerTable* peers, cudaStream_t s)
+{
+    return vec ? launch_reduce_t<true, BF, PEER>(grads, out, nd, segs, peers, s)
+               : launch_reduce_t<false, BF, PEER>(grads, out, nd, segs, peers, s);
+}
+
+cudaError_t launch_reduce(bool vec, bool bf16, const uint16_t* grads, uint16_t* out, int nd, const SegList& segs,
+                          const PeerTable* peers, cudaStream_t s)
+{
+    if (peers)
+        return bf16 ? launch_reduce_f<true, true>(vec, grads, out, nd, segs, peers, s)
+                    : launch_reduce_f<false, true>(vec, grads, out, nd, segs, peers, s);
+    return bf16 ? launch_reduce_f<true, false>(vec, grads, out, nd, segs, peers, s)
+                : launch_reduce_f<false, false>(vec, grads, out, nd, segs, peers, s);
 }
 
 template <bool VEC, bool BF>

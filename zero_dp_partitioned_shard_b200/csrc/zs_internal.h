@@ -157,5 +157,8 @@ cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bo
 cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
                         cudaStream_t s);
 cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s);
+// out[seg.s_off + e] = 16-bit rounding of the rank-order sum of nd contributions
+cudaError_t launch_reduce(bool vec, bool bf16, const uint16_t* grads, uint16_t* out, int nd, const SegList& segs,
+                          const PeerTable* peers, cudaStream_t s);
 
 } // namespace zs
