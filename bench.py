@@ -22,6 +22,11 @@ in this GPU's memory: each rank's gradient read through the table, every new
 parameter stored into all Nd full parameter buffers (the all-gather by
 stores), which adds 2 (Nd - 1) bytes per parameter.
 
+``--retain`` runs the stage-2 variant with gradient retention: per step the
+reduce-scatter keeps the owners' reduced gradients in 16 bits
+(``zero_reduce_scatter``, 2 Nd + 2 bytes per parameter) and the step reads
+that kept shard as its one contribution (28 bytes per parameter).
+
 Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): the path has
 no data exchange on one GPU, so N ranks run independent replicas (weak
 scaling); the only collectives are the timing barrier and the max over ranks.
@@ -174,7 +179,8 @@ class ClockSampler:
 class Bench:
     """Device buffers and the C-ABI arguments of one workload on one GPU."""
 
-    def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0, peer: bool = False):
+    def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0, peer: bool = False,
+                 retain: bool = False):
         import torch
         from zero_dp_partitioned_shard_b200 import binding as B
         from zero_dp_partitioned_shard_b200 import synth
@@ -256,6 +262,21 @@ class Bench:
             self.dests = [torch.zeros(psi, dtype=h16, device=dev) for _ in range(self.nd - 1)]
             rank_grads = [self.grads.data_ptr() + 2 * r * stride for r in range(self.nd)]
             B.attach_peers(self.args, B.peer_args(rank_grads, [t.data_ptr() for t in self.dests]))
+        # stage-2 retention: the reduce-scatter reads the contributions, the
+        # step reads the owners' kept 16-bit shards
+        self.retain_args, self.kept = None, None
+        if retain:
+            if peer or wl.get("assemble"):
+                raise ValueError("--retain runs the plain stage-2 layouts")
+            self.kept = torch.empty(n_state, dtype=h16, device=dev)
+            self.retain_args = B.step_args(
+                grads=self.grads.data_ptr(), grad_rank_stride=stride, grad_layout=wl["layout"],
+                owner_first=o0, owner_count=oc, master=(0, 0), exp_avg=(0, 0), exp_avg_sq=(0, 0),
+                params=0, opt_state=0, storage=storage)
+            self.args.grads = self.kept.data_ptr()
+            self.args.grad_layout = B.ZERO_GRADS_REDUCED
+            self.args.grad_rank_stride = 0
+            self.reduce_events = None
         ws_bytes = B.zero_workspace_bytes(self.plan, self.hp, self.args)
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.args.workspace = self.workspace.data_ptr()
@@ -270,6 +291,12 @@ class Bench:
         else:
             self.args.timing_events[0] = None
             self.args.timing_events[1] = None
+        if self.retain_args is not None:
+            if events is not None and len(events) > 2:
+                events[2].record()
+            self.B.zero_reduce_scatter(self.plan, self.retain_args, self.kept.data_ptr(), -1, self.stream)
+            if events is not None and len(events) > 2:
+                events[3].record()
         self.B.zero_shard_step(self.plan, self.hp, self.args, self.stream)
         if self.shard_ptrs is not None:
             self.B.zero_gather_params(self.plan, self.shard_ptrs, self.params.data_ptr(), self.stream)
@@ -478,6 +505,8 @@ def main():
                     help="16-bit format of gradients and parameters")
     ap.add_argument("--peer", action="store_true",
                     help="through peer tables, storing the parameters into all Nd ranks' buffers")
+    ap.add_argument("--retain", action="store_true",
+                    help="stage-2 retention: reduce-scatter into kept 16-bit shards, then the step on them")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -505,18 +534,20 @@ def main():
     import torch
     from zero_dp_partitioned_shard_b200 import binding as B
     world, rank, local = _dist()
-    bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage], peer=args.peer)
+    bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage], peer=args.peer,
+                  retain=args.retain)
     n_dests = len(bench.dests)
+    k_nd = 1 if args.retain else wl["nd"]          # contributions the update kernel reads
     alg, moved = bytes_per_param(wl["nd"], wl["mode"])
 
     # --- device-resident timing ---
     for _ in range(args.warmup):
         bench.step()
-    k_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-    for a, b in k_events:   # create the CUDA events before handing their handles over
-        a.record()
-        b.record()
+    n_ev = 4 if args.retain else 2
+    k_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(n_ev)) for _ in range(args.steps)]
+    for evs in k_events:    # create the CUDA events before handing their handles over
+        for ev in evs:
+            ev.record()
     torch.cuda.synchronize()
     _barrier(world)
     torch.cuda.synchronize()
@@ -535,7 +566,8 @@ def main():
     _barrier(world)
     ms = t_start.elapsed_time(t_end)
     ms_max, value = aggregate(bench.owned, args.steps, ms, world)
-    k_ms = statistics.mean(a.elapsed_time(b) for a, b in k_events)
+    k_ms = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in k_events)
+    r_ms = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in k_events) if args.retain else None
     k_ms_max = max_over_ranks(k_ms, world)
     res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
 
@@ -571,9 +603,10 @@ def main():
             e2e = {"value": None, "unit": UNIT, "skipped": "host memory below 2.5x the gradient bytes"}
 
     peak, peak_kind = measured_hbm_peak()
-    k_bytes = bench.owned * update_launch_bytes(wl["nd"], wl["mode"], n_dests)
+    k_bytes = bench.owned * update_launch_bytes(k_nd, wl["mode"], n_dests)
     achieved = k_bytes / (k_ms_max / 1e3) / 1e9
-    traffic, traffic_src = profiled_traffic(wl["nd"], wl["mode"], bench.owned) if not n_dests else (None, None)
+    traffic, traffic_src = (profiled_traffic(wl["nd"], wl["mode"], bench.owned)
+                            if not (n_dests or args.retain) else (None, None))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -581,6 +614,7 @@ def main():
         "config": {"workload": args.workload, "description": wl["desc"], "psi": bench.psi,
                    "nd": wl["nd"], "stage": wl["stage"], "storage": args.storage,
                    "peer_tables": bool(n_dests), "param_dests": n_dests,
+                   "retention": bool(args.retain),
                    "owned_params_per_gpu": bench.owned,
                    "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
                    "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
@@ -600,6 +634,13 @@ def main():
         "clocks": clk,
         "last_step": {"overflow": res.overflow, "t": res.t},
     }
+    if args.retain:
+        r_ms_max = max_over_ranks(r_ms, world)
+        line["retention"] = {"reduce_kernel_ms": r_ms_max, "reduce_bytes_per_param": 2 * wl["nd"] + 2,
+                             "reduce_gbs": bench.owned * (2 * wl["nd"] + 2) / (r_ms_max / 1e3) / 1e9}
+        line["retention"]["reduce_frac"] = line["retention"]["reduce_gbs"] / peak
+        line["config"]["step_gbs_alg"] = (bench.owned * (2 * wl["nd"] + 2 + update_launch_bytes(1, wl["mode"]))
+                                          / (ms_max / args.steps / 1e3) / 1e9)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.cpu_sample,
