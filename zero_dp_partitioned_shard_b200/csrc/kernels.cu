@@ -315,6 +315,8 @@ __device__ __forceinline__ void advance_loss_scale(zero_opt_state* st, bool skip
     }
 }
 
+// The clip coefficient is 1 when the step has no pre-pass (speculative): the
+// update kernels then skip the multiply by it, which would change no value.
 __device__ __forceinline__ AdamK load_consts(const UpdateArgs& a, const WsHeader* ws, bool clip)
 {
     AdamK k;
@@ -392,7 +394,7 @@ __device__ __forceinline__ bool update_scalar(const UpdateArgs& a, const PeerPar
     else
         g = __fmul_rn(rank_sum1<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd), inv);
     float p = p_in[so], m = m_in[so], v = v_in[so];
-    adam_update(__fmul_rn(g, k.clip), p, m, v, k);
+    adam_update(SRC == kSrcGradsSpeculative ? g : __fmul_rn(g, k.clip), p, m, v, k);
     p_out[so] = p;
     m_out[so] = m;
     v_out[so] = v;
@@ -447,7 +449,7 @@ zs_update_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, const
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                adam_update(__fmul_rn(g[q], k.clip), p[q], m[q], v[q], k);
+                adam_update(kSpec ? g[q] : __fmul_rn(g[q], k.clip), p[q], m[q], v[q], k);
             st_f8(p_out + so, p);
             st_f8(m_out + so, m);
             st_f8(v_out + so, v);
@@ -758,7 +760,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 }
 #pragma unroll
                 for (int q = 0; q < EPT; ++q)
-                    adam_update(__fmul_rn(gr[q], k.clip), p[q], m[q], v[q], k);
+                    adam_update(kSpec ? gr[q] : __fmul_rn(gr[q], k.clip), p[q], m[q], v[q], k);
                 const int64_t so = sg.s_off + e0 + i0;
                 stg_f<EPT>(p_out + so, p);
                 stg_f<EPT>(m_out + so, m);
