@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from _util import assert_f16_close, assert_f32_close
+from _util import assert_bf16_close, assert_f16_close, assert_f32_close
 from zero_dp_partitioned_shard_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
@@ -76,17 +76,27 @@ def _opt(bn):
     return B.opt_state_from_bytes(bn.opt_state.cpu().numpy().tobytes())
 
 
+def _kept_of(G, storage):
+    """The oracle's retained 16-bit reduction of sampled columns G [nd, k]."""
+    nd, k = G.shape
+    p = oracle.plan(k, nd, 1)
+    kept = oracle.reduce_scatter16(G, p, storage)
+    return np.concatenate([kept[o, :p.shard(o)[1]] for o in range(nd)])
+
+
 def _check_sampled_steps(bn, steps, n_random, seed, clip_from_gpu=False):
     lo, hi = bn.o0 * bn.L, bn.o0 * bn.L + bn.owned
     pos = _sample_positions(lo, hi, bn.L, bn.wl["bucket"], n_random, seed)
     G, idx = _gather_inputs(bn, pos)
+    if bn.kept is not None:            # retention: the step reads the kept reduction
+        G = _kept_of(G, bn.storage)[None, :]
     spec = bn.wl["mode"] == B.ZERO_MODE_SPECULATIVE
     slot = _opt(bn).cur if spec else 0
     master, m, v = _state_at(bn, idx, slot)
     P = _params_at(bn, idx)
     hp = oracle.HP(lr=bn.hp.lr, beta1=bn.hp.beta1, beta2=bn.hp.beta2, eps=bn.hp.eps,
                    weight_decay=bn.hp.weight_decay, loss_scale=bn.hp.loss_scale,
-                   max_grad_norm=bn.hp.max_grad_norm)
+                   max_grad_norm=bn.hp.max_grad_norm, storage=bn.storage)
     opt = oracle.Opt(*(lambda o: (o.t, o.beta1_pow, o.beta2_pow))(_opt(bn)))
     results = []
     for _ in range(steps):
@@ -105,7 +115,11 @@ def _check_sampled_steps(bn, steps, n_random, seed, clip_from_gpu=False):
     assert_f32_close(gm, master, 2, "master")
     assert_f32_close(ga, m, 2, "exp_avg")
     assert_f32_close(gv, v, 2, "exp_avg_sq")
-    assert_f16_close(_params_at(bn, idx), P, 1, "params")
+    close16 = assert_bf16_close if bn.storage == B.ZERO_STORAGE_BF16 else assert_f16_close
+    close16(_params_at(bn, idx), P, 1, "params")
+    for d, dst in enumerate(bn.dests):   # peer tables: every rank's buffer holds the same parameters
+        got = dst.view(torch.int16)[idx + bn.o0 * bn.L].cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, _params_at(bn, idx)), f"destination {d}"
     assert _opt(bn).t == opt.t
     return results
 
@@ -136,6 +150,43 @@ def test_gpt2_1p5b_stage2_nd8_speculative_sampled():
         for a, b in zip(before[0], after[0]):
             assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
         assert np.array_equal(before[1], after[1])
+    finally:
+        bn.close()
+
+
+def test_gpt2_1p5b_bf16_storage_sampled():
+    """The benchmark workload with bfloat16 gradients and parameters."""
+    bn = bench.Bench(_wl("gpt2-1.5b-stage2-nd8"), None, seed=6, storage=B.ZERO_STORAGE_BF16)
+    try:
+        assert bn.grads.dtype == torch.bfloat16
+        _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=6)
+    finally:
+        bn.close()
+
+
+def test_gpt2_1p5b_peer_tables_sampled():
+    """The benchmark workload through peer tables (bench --peer): the rank
+    contributions read through the table, every new parameter stored into all
+    8 ranks' buffers; each buffer checked at the sampled positions."""
+    bn = bench.Bench(_wl("gpt2-1.5b-stage2-nd8"), None, seed=7, peer=True)
+    try:
+        assert len(bn.dests) == 7
+        _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=7)
+    finally:
+        bn.close()
+
+
+def test_gpt2_1p5b_retention_sampled():
+    """The benchmark workload with stage-2 retention (bench --retain): the kept
+    fp16 reduction equals the oracle's bit for bit at the sampled positions,
+    and the step on it matches the oracle's step on the same kept values."""
+    bn = bench.Bench(_wl("gpt2-1.5b-stage2-nd8"), None, seed=8, retain=True)
+    try:
+        _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=8)
+        pos = _sample_positions(0, bn.owned, bn.L, bn.wl["bucket"], 1 << 18, 9)
+        G, idx = _gather_inputs(bn, pos)
+        got = bn.kept.view(torch.int16)[idx].cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, _kept_of(G, bn.storage))
     finally:
         bn.close()
 
