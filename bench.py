@@ -22,6 +22,15 @@ in this GPU's memory: each rank's gradient read through the table, every new
 parameter stored into all Nd full parameter buffers (the all-gather by
 stores), which adds 2 (Nd - 1) bytes per parameter.
 
+``--dynamic-scale`` keeps the loss scale in the device optimizer state
+(dynamic loss scaling) instead of the hyper-parameters; the step's bytes do
+not change.
+
+``--layer-gather`` measures the stage-3 schedule instead: the GPT-2
+1.5B-shaped tensor list at Nd = 8, every layer gathered from the owners'
+fp16 shards into a compact buffer while the previous one is in use, forward
+then backward (2 Psi elements gathered per pass pair, 4 bytes each).
+
 ``--retain`` runs the stage-2 variant with gradient retention: per step the
 reduce-scatter keeps the owners' reduced gradients in 16 bits
 (``zero_reduce_scatter``, 2 Nd + 2 bytes per parameter) and the step reads
@@ -180,7 +189,7 @@ class Bench:
     """Device buffers and the C-ABI arguments of one workload on one GPU."""
 
     def __init__(self, wl: dict, psi_override: int | None, seed: int, storage: int = 0, peer: bool = False,
-                 retain: bool = False):
+                 retain: bool = False, dynamic_scale: bool = False):
         import torch
         from zero_dp_partitioned_shard_b200 import binding as B
         from zero_dp_partitioned_shard_b200 import synth
@@ -230,7 +239,10 @@ class Bench:
                            storage=storage)
         self.opt_state = torch.zeros(B.OPT_STATE_BYTES, dtype=torch.uint8, device=dev)
         self.result = torch.zeros(B.RESULT_BYTES, dtype=torch.uint8, device=dev)
-        B.zero_opt_state_init(self.opt_state.data_ptr(), stream)
+        if dynamic_scale:    # the loss scale lives in the device optimizer state
+            B.zero_opt_state_init_dynamic(self.opt_state.data_ptr(), wl["S"], 2.0, 0.5, 2000, stream)
+        else:
+            B.zero_opt_state_init(self.opt_state.data_ptr(), stream)
         self.hp = B.hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"],
                             loss_scale=wl["S"], max_grad_norm=wl["clip"], mode=wl["mode"])
         ptr = lambda t: t.data_ptr() if t is not None else 0
@@ -489,6 +501,88 @@ def run_sweep(args) -> int:
     return 0
 
 
+def run_layer_gather(args) -> int:
+    """Stage-3 on-demand gathering: forward + backward passes of the per-layer
+    schedule over the GPT-2 1.5B-shaped tensor list at Nd = 8 (one JSON line,
+    measurement mode)."""
+    import torch
+    from zero_dp_partitioned_shard_b200 import binding as B
+    from zero_dp_partitioned_shard_b200 import synth
+    from zero_dp_partitioned_shard_b200.stage3 import LayerGatherSchedule
+    world, rank, local = _dist()
+    sizes = synth.gpt2_xl_tensor_sizes()
+    psi, nd = sum(sizes), 8
+    plan = B.zero_plan(psi, nd, stage=3, align_elems=256, tensor_sizes=sizes)
+    try:
+        L = B.zero_plan_query(plan).shard_len
+        shards = torch.empty(nd, L, dtype=torch.float16, device="cuda")
+        for o in range(nd):
+            synth.fill_normal_(shards[o], seed=600 + o, std=0.02)
+        per_layer = 12                                   # LN1, QKV, proj, LN2, MLP up and down (+ biases)
+        n_layer = (len(sizes) - 4) // per_layer
+        layers = [(i * per_layer, per_layer) for i in range(n_layer)] + [(n_layer * per_layer, 4)]
+        sched = LayerGatherSchedule(plan, layers, [shards[o].data_ptr() for o in range(nd)], sizes)
+        use = lambda layer, params: None                 # no model: the data movement alone
+        for _ in range(args.warmup):
+            sched.forward(use)
+            sched.backward(use)
+        torch.cuda.synchronize()
+        # the same passes recorded once as CUDA graphs (one launch per pass)
+        graphs = [sched.capture(range(len(layers)), use), sched.capture(reversed(range(len(layers))), use)]
+        for _ in range(args.warmup):
+            for gr in graphs:
+                gr.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(args.steps):
+            for gr in graphs:
+                gr.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(g0.elapsed_time(g1), world)
+        del graphs
+        _barrier(world)
+        clocks = ClockSampler(local)
+        clocks.start()
+        time.sleep(0.3)
+        gathered0 = sched.gathered
+        launches0 = B.zero_launch_count()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            sched.forward(use)
+            sched.backward(use)
+        e1.record()
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        ms = max_over_ranks(e0.elapsed_time(e1), world)
+        elems = (sched.gathered - gathered0) * world
+        peak, peak_kind = measured_hbm_peak()
+        gbs = elems * 4 / (ms / 1e3) / 1e9
+        if rank == 0:
+            print(json.dumps({
+                "mode": "layer_gather", "metric": "stage-3 gathered fp16 parameters per second",
+                "value": elems / (ms / 1e3), "unit": "params/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+                "config": {"workload": "gpt2-1.5b-stage3-nd8-layers", "psi": psi, "nd": nd, "layers": len(layers),
+                           "step": "forward + backward pass of the gather schedule (2 Psi elements)",
+                           "bytes_per_param": 4},
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                             "peak_source": f"{peak_kind} hbm_gbs (copy)"},
+                "gpu_launches": B.zero_launch_count() - launches0, "clocks": clk,
+                "graph_replay": {"ms_per_step": graph_ms / args.steps,
+                                 "value": elems / (graph_ms / 1e3),
+                                 "frac": elems * 4 / (graph_ms / 1e3) / 1e9 / peak}}), flush=True)
+        del sched, shards
+    finally:
+        B.zero_plan_destroy(plan)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def _psi_of(wl):
     return sum(wl["sizes"]()) if wl.get("sizes") else wl["psi"]
 
@@ -505,6 +599,10 @@ def main():
                     help="16-bit format of gradients and parameters")
     ap.add_argument("--peer", action="store_true",
                     help="through peer tables, storing the parameters into all Nd ranks' buffers")
+    ap.add_argument("--dynamic-scale", action="store_true",
+                    help="dynamic loss scaling (the scale in the device optimizer state)")
+    ap.add_argument("--layer-gather", action="store_true",
+                    help="measure the stage-3 per-layer gather schedule (forward + backward)")
     ap.add_argument("--retain", action="store_true",
                     help="stage-2 retention: reduce-scatter into kept 16-bit shards, then the step on them")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -524,6 +622,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.sweep:
         return run_sweep(args)
+    if args.layer_gather:
+        return run_layer_gather(args)
     wls = _workloads()
     if args.workload not in wls:
         ap.error(f"unknown workload {args.workload}; choose from {sorted(wls)}")
@@ -535,7 +635,7 @@ def main():
     from zero_dp_partitioned_shard_b200 import binding as B
     world, rank, local = _dist()
     bench = Bench(wl, args.psi or None, seed=1 + rank, storage=STORAGES[args.storage], peer=args.peer,
-                  retain=args.retain)
+                  retain=args.retain, dynamic_scale=args.dynamic_scale)
     n_dests = len(bench.dests)
     k_nd = 1 if args.retain else wl["nd"]          # contributions the update kernel reads
     alg, moved = bytes_per_param(wl["nd"], wl["mode"])
@@ -614,7 +714,7 @@ def main():
         "config": {"workload": args.workload, "description": wl["desc"], "psi": bench.psi,
                    "nd": wl["nd"], "stage": wl["stage"], "storage": args.storage,
                    "peer_tables": bool(n_dests), "param_dests": n_dests,
-                   "retention": bool(args.retain),
+                   "retention": bool(args.retain), "dynamic_loss_scale": bool(args.dynamic_scale),
                    "owned_params_per_gpu": bench.owned,
                    "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[wl["mode"]],
                    "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,

@@ -99,3 +99,46 @@ def test_layer_schedule_forward_backward_and_volume():
         assert sched.gathered + psi == oracle.state_bytes(psi, nd, 3)["comm_elems"]
     finally:
         B.zero_plan_destroy(plan)
+
+
+def test_layer_schedule_graph_replay_matches_eager():
+    """The forward + backward passes captured once as a CUDA graph: each
+    replay gathers every layer again (the shards change between replays),
+    and each layer equals the oracle's gather of the current shards."""
+    n_layer, d = 5, 64
+    sizes = synth.transformer_tensor_sizes(n_layer, d, 500, 32)
+    psi, nd = sum(sizes), 4
+    p = oracle.plan(psi, nd, 8)
+    layers = [(12 * i, 12) for i in range(n_layer)] + [(12 * n_layer, 4)]
+    plan = B.zero_plan(psi, nd, stage=3, align_elems=8, tensor_sizes=sizes)
+    try:
+        ref = synth.fp16_bits(synth.normal_f32(psi, seed=21, std=0.02))
+        host_sh, dev_sh = _shards(p, ref)
+        sched = stage3.LayerGatherSchedule(plan, layers, [t.data_ptr() for t in dev_sh], sizes)
+        cap = max(sched.sizes)
+        outs = {pas: torch.zeros(len(layers), cap, dtype=torch.float16, device="cuda") for pas in ("fwd", "bwd")}
+        fwd = lambda i, w: outs["fwd"][i, :w.numel()].copy_(w)
+        bwd = lambda i, w: outs["bwd"][i, :w.numel()].copy_(w)
+        sched.forward(fwd)                       # eager first: caches and launch geometry
+        sched.backward(bwd)
+        g_fwd = sched.capture(range(len(layers)), fwd)
+        g_bwd = sched.capture(reversed(range(len(layers))), bwd)
+        for seed in (22, 23):
+            ref = synth.fp16_bits(synth.normal_f32(psi, seed=seed, std=0.02))
+            new_host, new_dev = _shards(p, ref)
+            for r in range(nd):              # same device buffers, new contents
+                dev_sh[r].copy_(new_dev[r])
+            outs["fwd"].zero_()
+            outs["bwd"].zero_()
+            g_fwd.replay()
+            g_bwd.replay()
+            torch.cuda.synchronize()
+            for pas in ("fwd", "bwd"):
+                got = outs[pas].cpu().numpy().view(np.uint16)
+                for i, (first, count) in enumerate(layers):
+                    want = np.zeros(psi, np.uint16)
+                    n = oracle.gather_tensors(new_host, p, sizes, first, count, want, True)
+                    assert np.array_equal(got[i, :n], want[:n]), (seed, pas, i)
+        del g_fwd, g_bwd
+    finally:
+        B.zero_plan_destroy(plan)

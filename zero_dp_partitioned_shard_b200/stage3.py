@@ -73,3 +73,18 @@ class LayerGatherSchedule:
 
     def backward(self, use) -> None:
         self.run(reversed(range(len(self.layers))), use)
+
+    def capture(self, order, use) -> torch.cuda.CUDAGraph:
+        """Records ``run(order, use)`` once as a CUDA graph: every layer's
+        gather, the side-stream prefetch and the release ordering become
+        graph nodes, and ``replay()`` re-issues the whole pass with one launch
+        instead of a host round per layer.  ``use`` must be capturable (work
+        enqueued on the current stream, no host synchronisation).  The
+        schedule's buffers stay the graph's: do not run the schedule eagerly
+        while a replay may be in flight.  Replays do not add to
+        ``gathered``; the capture counts one pass."""
+        graph = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize(self.device)
+        with torch.cuda.graph(graph):
+            self.run(order, use)
+        return graph
