@@ -14,6 +14,9 @@ upskillscore.com, "How it works").
 ``zero_gather_tensors``: two compact layer buffers, the next layer's gather
 issued on a side stream while the current layer is in use (prefetch), and a
 buffer reused only after the work that used it has finished (release).
+Consecutive gathers fill different buffers and only read the shards, so each
+buffer has its own copy stream and one gather's tail overlaps the next one's
+start.
 """
 from __future__ import annotations
 
@@ -35,15 +38,16 @@ class LayerGatherSchedule:
         self.device = dev
         cap = max(self.sizes) if self.sizes else 1
         self.buffers = [torch.empty(cap, dtype=torch.float16, device=dev) for _ in range(2)]
-        self.copy_stream = torch.cuda.Stream(dev)
+        self.copy_streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]   # one per buffer
         self.gathered = 0   # elements gathered so far (the communication volume)
 
     def _issue(self, layer: int, slot: int, free: torch.cuda.Event, ready: torch.cuda.Event) -> None:
         first, count = self.layers[layer]
-        self.copy_stream.wait_event(free)             # the slot's last use has finished
+        cs = self.copy_streams[slot]
+        cs.wait_event(free)                           # the slot's last use has finished
         n = B.zero_gather_tensors(self.plan, first, count, self.shard_ptrs,
-                                  self.buffers[slot].data_ptr(), True, self.copy_stream.cuda_stream)
-        ready.record(self.copy_stream)
+                                  self.buffers[slot].data_ptr(), True, cs.cuda_stream)
+        ready.record(cs)
         self.gathered += n
 
     def run(self, order, use) -> None:
@@ -66,7 +70,8 @@ class LayerGatherSchedule:
             main.wait_event(ready[slot])
             use(layer, self.buffers[slot][:self.sizes[layer]])
             free[slot].record(main)                   # release after use
-        main.wait_stream(self.copy_stream)
+        for cs in self.copy_streams:
+            main.wait_stream(cs)
 
     def forward(self, use) -> None:
         self.run(range(len(self.layers)), use)
