@@ -497,16 +497,17 @@ zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hparams* hp,
     return run_step(plan, hp, args, stream, PHASE_END);
 }
 
-// Launches copies of shard pieces, at most kMaxSegs per launch.
-static zero_status launch_pieces(std::vector<zs::GatherEntry>& entries, uint16_t* dst, cudaStream_t str,
-                                 const char* what)
+// Launches copies of shard pieces, at most kMaxSegs per launch; compact
+// (small, reused layer buffers) copies use evict-first stores.
+static zero_status launch_pieces(std::vector<zs::GatherEntry>& entries, uint16_t* dst, bool compact,
+                                 cudaStream_t str, const char* what)
 {
     for (size_t i = 0; i < entries.size(); i += zs::kMaxSegs) {
         zs::GatherList g;
         std::memset(&g, 0, sizeof g);
         for (size_t k = i; k < entries.size() && g.count < zs::kMaxSegs; ++k)
             g.e[g.count++] = entries[k];
-        cudaError_t e = zs::launch_gather(dst, g, str);
+        cudaError_t e = zs::launch_gather(dst, g, compact, str);
         if (e != cudaSuccess)
             return cuda_fail(e, what);
     }
@@ -541,7 +542,7 @@ zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard
         if (n > 0)
             entries.push_back(piece(shard_ptrs[r], 0, params_full, start, n));
     }
-    return launch_pieces(entries, static_cast<uint16_t*>(params_full), static_cast<cudaStream_t>(stream),
+    return launch_pieces(entries, static_cast<uint16_t*>(params_full), false, static_cast<cudaStream_t>(stream),
                          "gather launch");
 }
 
@@ -585,7 +586,7 @@ zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, i
     }
     if (elements)
         *elements = n_elems;
-    return launch_pieces(entries, static_cast<uint16_t*>(out), static_cast<cudaStream_t>(stream),
+    return launch_pieces(entries, static_cast<uint16_t*>(out), compact != 0, static_cast<cudaStream_t>(stream),
                          "gather launch");
 }
 

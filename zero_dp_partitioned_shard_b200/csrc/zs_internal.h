@@ -156,7 +156,9 @@ cudaError_t launch_commit(bool vec, const UpdateArgs& a, const SegList& segs, bo
                           zero_opt_state* st, zero_step_result* res, const PeerTable* peers, cudaStream_t s);
 cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
                         cudaStream_t s);
-cudaError_t launch_gather(uint16_t* dst, const GatherList& g, cudaStream_t s);
+// streaming_stores: evict-first stores (compact per-layer buffers) or plain
+// ones (a full parameter buffer)
+cudaError_t launch_gather(uint16_t* dst, const GatherList& g, bool streaming_stores, cudaStream_t s);
 // out[seg.s_off + e] = 16-bit rounding of the rank-order sum of nd contributions
 cudaError_t launch_reduce(bool vec, bool bf16, const uint16_t* grads, uint16_t* out, int nd, const SegList& segs,
                           const PeerTable* peers, cudaStream_t s);
