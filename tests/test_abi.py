@@ -369,3 +369,59 @@ def test_gather_tensors_validation():
     finally:
         B.zero_plan_destroy(no_list)
         B.zero_plan_destroy(with_list)
+
+
+_C_CALLER = r"""
+/* A plain C caller of libzero_shard.so: host-only entry points and the
+ * checks that reject a step before anything is launched. */
+#include <stdio.h>
+#include <string.h>
+#include "zero_shard.h"
+#define CHECK(c) do { if (!(c)) { printf("FAIL line %d\n", __LINE__); return 1; } } while (0)
+int main(void) {
+    CHECK(zero_abi_version() == ZERO_SHARD_ABI_VERSION);
+    /* the pages' 7.5B / Nd = 64 example, stage 3: 1.875 GB per device, 3 Psi moved */
+    zero_state_report r;
+    CHECK(zero_state_bytes(7500000000LL, 64, 3, 1, &r) == ZERO_OK);
+    CHECK(r.total_bytes == 1.875e9 && r.comm_elems == 3 * 7.5e9);
+    /* the GPT-2 1.5B-shaped plan at Nd = 8 */
+    zero_plan_desc d;
+    memset(&d, 0, sizeof d);
+    d.psi = 1557611200; d.nd = 8; d.stage = 2; d.align_elems = 256;
+    zero_plan_t* plan = NULL;
+    CHECK(zero_plan(&d, &plan) == ZERO_OK && plan);
+    zero_plan_info info;
+    CHECK(zero_plan_query(plan, &info) == ZERO_OK);
+    CHECK(info.shard_len == 194701568 && info.psi_pad == 8 * 194701568LL);
+    int64_t start = 0, len = 0;
+    CHECK(zero_plan_shard(plan, 7, &start, &len) == ZERO_OK && start == 7 * 194701568LL && len == 194700224);
+    /* a step with no buffers is refused before any launch */
+    zero_hparams hp;
+    memset(&hp, 0, sizeof hp);
+    hp.loss_scale = 1.0f; hp.beta1 = 0.9f; hp.beta2 = 0.999f;
+    zero_step_args a;
+    memset(&a, 0, sizeof a);
+    a.owner_count = 8; a.grad_rank_stride = info.psi_pad;
+    const uint64_t before = zero_launch_count();
+    CHECK(zero_shard_step(plan, &hp, &a, NULL) == ZERO_ERR_INVALID_ARG);
+    CHECK(strlen(zero_last_error()) > 0);
+    CHECK(zero_launch_count() == before);
+    CHECK(strcmp(zero_strerror(ZERO_ERR_UNSUPPORTED), zero_strerror(ZERO_OK)) != 0);
+    zero_plan_destroy(plan);
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_plain_c_caller_links_and_calls_the_library(tmp_path):
+    """The ABI from C, not only through ctypes: a C program includes the
+    header, links libzero_shard.so and calls its host-side entry points."""
+    src = tmp_path / "caller.c"
+    src.write_text(_C_CALLER)
+    exe = tmp_path / "caller"
+    pkg = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", pkg, "-lzero_shard", "-Wl,-rpath," + pkg], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
