@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from _gpu import PARAM_SENTINEL, dev, host, make_problem, run_gpu, to_oracle_hp
-from _util import assert_f16_close, assert_f32_close
+from _util import assert_bf16_close, assert_f16_close, assert_f32_close
 from zero_dp_partitioned_shard_b200 import binding as B
 
 pytestmark = pytest.mark.gpu
@@ -148,36 +148,39 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_zero_dp_step_over_an_nccl_group():
+@pytest.mark.parametrize("storage", [B.ZERO_STORAGE_FP16, B.ZERO_STORAGE_BF16], ids=["fp16", "bf16"])
+def test_zero_dp_step_over_an_nccl_group(storage):
     import torch.distributed as dist
     from zero_dp_partitioned_shard_b200 import distributed as D
     from zero_dp_partitioned_shard_b200 import synth
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
                             device_id=torch.device("cuda", torch.cuda.current_device()))
+    bf = storage == B.ZERO_STORAGE_BF16
     try:
         psi = 1_000_003
         hp = B.hparams(loss_scale=1024.0, weight_decay=0.01)
-        zs = D.ZeroDPStep(psi, hp, align=256)
+        zs = D.ZeroDPStep(psi, hp, align=256, storage=storage)
         master0 = synth.normal_f32(psi, seed=5, std=0.02)
         zs.load_master(torch.from_numpy(master0))
-        grads = [synth.grads_f16(1, psi, seed=60 + t, std=1e-3, scale=1024.0, stride=zs.psi_pad,
-                                 pad_fill=0.0)[0] for t in range(2)]
+        draw = synth.grads_bf16 if bf else synth.grads_f16
+        grads = [draw(1, psi, seed=60 + t, std=1e-3, scale=1024.0, stride=zs.psi_pad,
+                      pad_fill=0.0)[0] for t in range(2)]
         for G in grads:
-            zs.step(torch.from_numpy(G.view(np.float16)).cuda())
+            zs.step(torch.from_numpy(G.view(np.int16)).cuda().view(zs.dtype))
         torch.cuda.synchronize()
         master, m, v = (x.cpu().numpy()[:psi] for x in zs.live_state())
-        params = zs.params.cpu().numpy().view(np.uint16)[:psi]
+        params = zs.params.view(torch.int16).cpu().numpy().view(np.uint16)[:psi]
         res = B.step_result_from_bytes(zs.result.cpu().numpy().tobytes())
         zs.close()
     finally:
         dist.destroy_process_group()
     ref_master, ref_m, ref_v = master0.copy(), np.zeros(psi, np.float32), np.zeros(psi, np.float32)
-    ref_P = oracle.float_to_half(master0)
+    ref_P = oracle.float_to_bf16(master0) if bf else oracle.float_to_half(master0)
     opt = oracle.Opt()
     for G in grads:
         oracle.step(G[None, :psi].copy(), ref_master, ref_m, ref_v, ref_P,
-                    oracle.HP(loss_scale=1024.0, weight_decay=0.01), opt)
+                    oracle.HP(loss_scale=1024.0, weight_decay=0.01, storage=storage), opt)
     assert res.t == 2 and res.overflow == 0 and res.status == 0
     assert_f32_close(master, ref_master, 2, "master")
     assert_f32_close(v, ref_v, 2, "exp_avg_sq")
-    assert_f16_close(params, ref_P, 1, "params")
+    (assert_bf16_close if bf else assert_f16_close)(params, ref_P, 1, "params")

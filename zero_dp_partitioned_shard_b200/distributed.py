@@ -119,11 +119,13 @@ class ZeroDPStep:
     """
 
     def __init__(self, psi: int, hp: B.HParams, *, group=None, align: int = 256,
-                 bucket: int = 0, stage: int = 2, device=None):
+                 bucket: int = 0, stage: int = 2, device=None, storage: int = B.ZERO_STORAGE_FP16):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.hp = hp
+        self.storage = storage
+        self.dtype = torch.bfloat16 if storage == B.ZERO_STORAGE_BF16 else torch.float16
         self.plan = B.zero_plan(psi, self.world, stage=stage, align_elems=align, bucket_elems=bucket)
         info = B.zero_plan_query(self.plan)
         self.psi, self.L, self.psi_pad = psi, info.shard_len, info.psi_pad
@@ -135,8 +137,8 @@ class ZeroDPStep:
         self.exp_avg = [f32(), f32() if spec else None]
         self.exp_avg_sq = [f32(), f32() if spec else None]
         self.stash = f32() if hp.mode == B.ZERO_MODE_STASH else None
-        self.params = torch.zeros(self.psi_pad, dtype=torch.float16, device=dev)
-        self.recv = torch.zeros(self.psi_pad, dtype=torch.float16, device=dev)
+        self.params = torch.zeros(self.psi_pad, dtype=self.dtype, device=dev)
+        self.recv = torch.zeros(self.psi_pad, dtype=self.dtype, device=dev)
         self.opt_state = torch.zeros(B.OPT_STATE_BYTES, dtype=torch.uint8, device=dev)
         self.result = torch.zeros(B.RESULT_BYTES, dtype=torch.uint8, device=dev)
         ptr = lambda t: t.data_ptr() if t is not None else 0
@@ -145,7 +147,7 @@ class ZeroDPStep:
             owner_first=self.rank, owner_count=1, master=tuple(map(ptr, self.master)),
             exp_avg=tuple(map(ptr, self.exp_avg)), exp_avg_sq=tuple(map(ptr, self.exp_avg_sq)),
             params=self.params.data_ptr(), grad_stash=ptr(self.stash),
-            opt_state=self.opt_state.data_ptr(), result=self.result.data_ptr())
+            opt_state=self.opt_state.data_ptr(), result=self.result.data_ptr(), storage=storage)
         ws_bytes = B.zero_workspace_bytes(self.plan, hp, self.args)
         self.workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
         self.args.workspace = self.workspace.data_ptr()
@@ -159,18 +161,19 @@ class ZeroDPStep:
 
     def load_master(self, master_full: torch.Tensor) -> None:
         """Initialise this process's fp32 shard from the full fp32 master
-        (any device) and all-gather the fp16 cast into ``params``."""
+        (any device) and all-gather the 16-bit cast into ``params``."""
         s, n = B.zero_plan_shard(self.plan, self.rank)
         self.master[0].zero_()
         self.master[0][:n].copy_(master_full[s:s + n])
         B.zero_cast_params(self.plan, self.master[0].data_ptr(), self.params.data_ptr(), self.rank, 1,
-                           self._stream())
+                           self._stream(), storage=self.storage)
         gather_params(self.params, self.L, self.group)
 
     def step(self, grad_flat: torch.Tensor) -> torch.Tensor:
-        """One ZeRO-DP step from this process's local fp16 gradient (Nd*L
-        elements, pads zero).  Returns the device result struct (raw bytes)."""
-        assert grad_flat.dtype == torch.float16 and grad_flat.numel() == self.psi_pad
+        """One ZeRO-DP step from this process's local 16-bit gradient (Nd*L
+        elements, pads zero, the storage format's dtype).  Returns the device
+        result struct (raw bytes)."""
+        assert grad_flat.dtype == self.dtype and grad_flat.numel() == self.psi_pad
         stream = self._stream()
         exchange_gradients(grad_flat, self.recv, self.group)
         B.zero_shard_step_begin(self.plan, self.hp, self.args, stream)
