@@ -40,7 +40,10 @@
  * Conventions for every call:
  *   - Pointers documented "device" are CUDA device addresses on the device
  *     current when the call is made; "host" pointers are ordinary memory.
- *   - fp16 data is IEEE binary16 passed as void* / uint16_t bit patterns.
+ *   - 16-bit data (gradients, parameters) is IEEE binary16 by default, or
+ *     bfloat16 where a call's storage argument says so (ZERO_STORAGE_*),
+ *     passed as void* / uint16_t bit patterns.  Below, "fp16" names that
+ *     16-bit format.
  *   - The caller allocates and owns every device buffer (parameters, state,
  *     gradients, workspace).  The library allocates only the host-side plan
  *     object, never device memory, and never synchronises a stream.
