@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 6
+#define ZERO_SHARD_ABI_VERSION 7
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -488,6 +488,19 @@ ZERO_API zero_status zero_gather_params(const zero_plan_t* plan, const void* con
 ZERO_API zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
                                          const void* const* shard_ptrs, void* out, int32_t compact,
                                          int64_t* elements, void* stream);
+
+/* zero_gather_tensors moved by the GPU's copy engines instead of a kernel:
+ * the same pieces, arguments, results and errors, with one device-to-device
+ * cudaMemcpyAsync per run of pieces that continue each other in both the
+ * shard and the destination (the consecutive tensors one owner holds).  No
+ * SM runs the copy, so it proceeds beside kernels that occupy every SM on
+ * other streams (a layer's compute while the next layer is prefetched),
+ * where a copy kernel would wait for SMs; alone it is slower than the
+ * kernel.  Shards on other GPUs (mapped with zero_ipc_open) are reached the
+ * same way, over NVLink. */
+ZERO_API zero_status zero_gather_tensors_dma(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                             const void* const* shard_ptrs, void* out, int32_t compact,
+                                             int64_t* elements, void* stream);
 
 /* params[(owner_first + j) * L + i] = cast(master[j * L + i]) for the owners
  * owner_first .. owner_first + owner_count - 1, in the 16-bit format

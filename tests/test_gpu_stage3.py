@@ -33,8 +33,13 @@ def _shards(p, ref):
     return host_sh, dev_sh
 
 
+GATHERS = {"kernel": B.zero_gather_tensors, "dma": B.zero_gather_tensors_dma}
+
+
+@pytest.mark.parametrize("engine", sorted(GATHERS))
 @pytest.mark.parametrize("nd,align,seed", [(3, 1, 1), (8, 8, 2), (4, 256, 3), (16, 256, 4)])
-def test_gather_tensors_matches_oracle(nd, align, seed):
+def test_gather_tensors_matches_oracle(nd, align, seed, engine):
+    gather = GATHERS[engine]
     rs = np.random.default_rng(seed)
     sizes = [int(x) for x in rs.integers(1, 40_000, size=40)] + [7, 1600, 4800, 13]
     psi = sum(sizes)
@@ -48,8 +53,7 @@ def test_gather_tensors_matches_oracle(nd, align, seed):
             want = np.zeros(max(1, psi), np.uint16)
             n_ref = oracle.gather_tensors(host_sh, p, sizes, first, count, want, True)
             out = dev(np.full(max(1, n_ref) + 64, 0x7DDD, np.uint16))
-            n = B.zero_gather_tensors(plan, first, count, [t.data_ptr() for t in dev_sh],
-                                      out.data_ptr(), True, stream)
+            n = gather(plan, first, count, [t.data_ptr() for t in dev_sh], out.data_ptr(), True, stream)
             got = host(out)
             assert n == n_ref
             assert np.array_equal(got[:n], want[:n]) and (got[n:] == 0x7DDD).all()
@@ -60,18 +64,19 @@ def test_gather_tensors_matches_oracle(nd, align, seed):
         full_init[s0:s0 + n0] = ref[s0:s0 + n0]
         full = dev(full_init)
         ptrs = [0 if r == skip else dev_sh[r].data_ptr() for r in range(nd)]
-        B.zero_gather_tensors(plan, 2, len(sizes) - 5, ptrs, full.data_ptr(), False, stream)
+        gather(plan, 2, len(sizes) - 5, ptrs, full.data_ptr(), False, stream)
         want = full_init.copy()
         oracle.gather_tensors([None if r == skip else host_sh[r] for r in range(nd)], p, sizes,
                               2, len(sizes) - 5, want, False)
         assert np.array_equal(host(full), want)
         with pytest.raises(B.ZeroError):   # compact needs every owner's shard
-            B.zero_gather_tensors(plan, 0, len(sizes), ptrs, out.data_ptr(), True, stream)
+            gather(plan, 0, len(sizes), ptrs, out.data_ptr(), True, stream)
     finally:
         B.zero_plan_destroy(plan)
 
 
-def test_layer_schedule_forward_backward_and_volume():
+@pytest.mark.parametrize("engine", ["kernel", "dma"])
+def test_layer_schedule_forward_backward_and_volume(engine):
     n_layer, d = 6, 96
     sizes = synth.transformer_tensor_sizes(n_layer, d, 1000, 64)
     psi, nd = sum(sizes), 4
@@ -81,7 +86,7 @@ def test_layer_schedule_forward_backward_and_volume():
     layers = [(12 * i, 12) for i in range(n_layer)] + [(12 * n_layer, 4)]
     plan = B.zero_plan(psi, nd, stage=3, align_elems=8, tensor_sizes=sizes)
     try:
-        sched = stage3.LayerGatherSchedule(plan, layers, [t.data_ptr() for t in dev_sh], sizes)
+        sched = stage3.LayerGatherSchedule(plan, layers, [t.data_ptr() for t in dev_sh], sizes, engine=engine)
         seen = {"fwd": [], "bwd": []}
         sched.forward(lambda i, w: seen["fwd"].append((i, w.clone())))
         sched.backward(lambda i, w: seen["bwd"].append((i, w.clone())))
@@ -101,7 +106,8 @@ def test_layer_schedule_forward_backward_and_volume():
         B.zero_plan_destroy(plan)
 
 
-def test_layer_schedule_graph_replay_matches_eager():
+@pytest.mark.parametrize("engine", ["kernel", "dma"])
+def test_layer_schedule_graph_replay_matches_eager(engine):
     """The forward + backward passes captured once as a CUDA graph: each
     replay gathers every layer again (the shards change between replays),
     and each layer equals the oracle's gather of the current shards."""
@@ -114,7 +120,7 @@ def test_layer_schedule_graph_replay_matches_eager():
     try:
         ref = synth.fp16_bits(synth.normal_f32(psi, seed=21, std=0.02))
         host_sh, dev_sh = _shards(p, ref)
-        sched = stage3.LayerGatherSchedule(plan, layers, [t.data_ptr() for t in dev_sh], sizes)
+        sched = stage3.LayerGatherSchedule(plan, layers, [t.data_ptr() for t in dev_sh], sizes, engine=engine)
         cap = max(sched.sizes)
         outs = {pas: torch.zeros(len(layers), cap, dtype=torch.float16, device="cuda") for pas in ("fwd", "bwd")}
         fwd = lambda i, w: outs["fwd"][i, :w.numel()].copy_(w)

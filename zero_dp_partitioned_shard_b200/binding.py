@@ -144,6 +144,7 @@ SIGNATURES = {
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
     "zero_reduce_scatter": (_S, [_P, C.POINTER(StepArgs), C.c_int64, _P, _P]),
     "zero_gather_tensors": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
+    "zero_gather_tensors_dma": (_S, [_P, C.c_int32, C.c_int32, _P, _P, C.c_int32, C.POINTER(C.c_int64), _P]),
     "zero_cast_params": (_S, [_P, _P, _P, C.c_int32, C.c_int32, C.c_int32, _P]),
     "zero_ipc_export": (_S, [_P, C.POINTER(IpcHandle)]),
     "zero_ipc_open": (_S, [C.POINTER(IpcHandle), C.POINTER(_P)]),
@@ -169,7 +170,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 6:
+        if L.zero_abi_version() != 7:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -293,6 +294,16 @@ def zero_gather_tensors(plan: int, first_tensor: int, n_tensors: int, shard_ptrs
     n = C.c_int64()
     _check(lib().zero_gather_tensors(plan, first_tensor, n_tensors, C.cast(arr, C.c_void_p), out,
                                      int(compact), C.byref(n), stream), "zero_gather_tensors")
+    return n.value
+
+
+def zero_gather_tensors_dma(plan: int, first_tensor: int, n_tensors: int, shard_ptrs, out: int,
+                            compact: bool, stream: int = 0) -> int:
+    """zero_gather_tensors moved by the copy engines; returns the elements copied."""
+    arr = (C.c_void_p * len(shard_ptrs))(*[p if p else None for p in shard_ptrs])
+    n = C.c_int64()
+    _check(lib().zero_gather_tensors_dma(plan, first_tensor, n_tensors, C.cast(arr, C.c_void_p), out,
+                                         int(compact), C.byref(n), stream), "zero_gather_tensors_dma")
     return n.value
 
 

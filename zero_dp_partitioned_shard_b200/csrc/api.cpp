@@ -546,27 +546,26 @@ zero_status zero_gather_params(const zero_plan_t* plan, const void* const* shard
                          "gather launch");
 }
 
-zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
-                                const void* const* shard_ptrs, void* out, int32_t compact,
-                                int64_t* elements, void* stream)
+// The pieces (owner shard range -> destination offset) of a tensor range.
+static zero_status tensor_pieces(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                 const void* const* shard_ptrs, void* out, int32_t compact, const char* who,
+                                 std::vector<zs::GatherEntry>* entries, int64_t* n_elems)
 {
-    zs::clear_error();
     if (!plan || !shard_ptrs || !out)
-        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: null argument");
+        return fail(ZERO_ERR_INVALID_ARG, "%s: null argument", who);
     const zero_plan_s& p = *plan;
     const int32_t nt = (int32_t)p.tensor_offset.size() - 1;
     if (nt < 1)
-        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: the plan was built without a tensor list");
+        return fail(ZERO_ERR_INVALID_ARG, "%s: the plan was built without a tensor list", who);
     if (first_tensor < 0 || n_tensors < 0 || first_tensor > nt - n_tensors)
-        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: tensors [%d, %d + %d) outside [0, %d)",
+        return fail(ZERO_ERR_INVALID_ARG, "%s: tensors [%d, %d + %d) outside [0, %d)", who,
                     first_tensor, first_tensor, n_tensors, nt);
     if (compact != 0 && compact != 1)
-        return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: compact must be 0 or 1");
+        return fail(ZERO_ERR_INVALID_ARG, "%s: compact must be 0 or 1", who);
     if (!aligned(out, 2))
-        return fail(ZERO_ERR_ALIGNMENT, "zero_gather_tensors: out must be 2-byte aligned");
+        return fail(ZERO_ERR_ALIGNMENT, "%s: out must be 2-byte aligned", who);
     const int64_t base = p.tensor_offset[(size_t)first_tensor];
-    std::vector<zs::GatherEntry> entries;
-    int64_t n_elems = 0;
+    *n_elems = 0;
     for (const zero_segment& sg : p.segments) {
         if (sg.tensor < first_tensor || sg.tensor >= first_tensor + n_tensors)
             continue;
@@ -574,20 +573,65 @@ zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, i
         const int64_t flat = p.tensor_offset[(size_t)sg.tensor] + sg.offset_in_tensor;
         if (!sh) {
             if (compact)
-                return fail(ZERO_ERR_INVALID_ARG, "zero_gather_tensors: tensor %lld needs owner %lld's shard",
+                return fail(ZERO_ERR_INVALID_ARG, "%s: tensor %lld needs owner %lld's shard", who,
                             (long long)sg.tensor, (long long)sg.owner);
             continue; // in place: this owner's part is already there
         }
         if (!aligned(sh, 2))
-            return fail(ZERO_ERR_ALIGNMENT, "zero_gather_tensors: shard %lld must be 2-byte aligned",
-                        (long long)sg.owner);
-        entries.push_back(piece(sh, sg.offset_in_shard, out, compact ? flat - base : flat, sg.length));
-        n_elems += sg.length;
+            return fail(ZERO_ERR_ALIGNMENT, "%s: shard %lld must be 2-byte aligned", who, (long long)sg.owner);
+        entries->push_back(piece(sh, sg.offset_in_shard, out, compact ? flat - base : flat, sg.length));
+        *n_elems += sg.length;
     }
+    return ZERO_OK;
+}
+
+zero_status zero_gather_tensors(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                const void* const* shard_ptrs, void* out, int32_t compact,
+                                int64_t* elements, void* stream)
+{
+    zs::clear_error();
+    std::vector<zs::GatherEntry> entries;
+    int64_t n_elems = 0;
+    zero_status s = tensor_pieces(plan, first_tensor, n_tensors, shard_ptrs, out, compact, "zero_gather_tensors",
+                                  &entries, &n_elems);
+    if (s != ZERO_OK)
+        return s;
     if (elements)
         *elements = n_elems;
     return launch_pieces(entries, static_cast<uint16_t*>(out), compact != 0, static_cast<cudaStream_t>(stream),
                          "gather launch");
+}
+
+zero_status zero_gather_tensors_dma(const zero_plan_t* plan, int32_t first_tensor, int32_t n_tensors,
+                                    const void* const* shard_ptrs, void* out, int32_t compact,
+                                    int64_t* elements, void* stream)
+{
+    zs::clear_error();
+    std::vector<zs::GatherEntry> entries;
+    int64_t n_elems = 0;
+    zero_status s = tensor_pieces(plan, first_tensor, n_tensors, shard_ptrs, out, compact,
+                                  "zero_gather_tensors_dma", &entries, &n_elems);
+    if (s != ZERO_OK)
+        return s;
+    if (elements)
+        *elements = n_elems;
+    // pieces that continue each other in both the shard and the destination
+    // (consecutive tensors of one owner) move as one copy
+    uint16_t* dst = static_cast<uint16_t*>(out);
+    cudaStream_t str = static_cast<cudaStream_t>(stream);
+    for (size_t i = 0; i < entries.size();) {
+        const uint16_t* src = entries[i].src;
+        const int64_t off = entries[i].dst_off;
+        int64_t n = entries[i].n;
+        size_t j = i + 1;
+        while (j < entries.size() && entries[j].src == src + n && entries[j].dst_off == off + n)
+            n += entries[j++].n;
+        const cudaError_t e = cudaMemcpyAsync(dst + off, src, (size_t)n * 2, cudaMemcpyDeviceToDevice, str);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "zero_gather_tensors_dma copy");
+        i = j;
+    }
+    return ZERO_OK;
 }
 
 zero_status zero_cast_params(const zero_plan_t* plan, const float* master, void* params,

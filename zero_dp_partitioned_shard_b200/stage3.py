@@ -16,7 +16,9 @@ issued on a side stream while the current layer is in use (prefetch), and a
 buffer reused only after the work that used it has finished (release).
 Consecutive gathers fill different buffers and only read the shards, so each
 buffer has its own copy stream and one gather's tail overlaps the next one's
-start.
+start.  ``engine="dma"`` moves the layers with the copy engines
+(``zero_gather_tensors_dma``) instead of a copy kernel, so a gather can run
+beside compute that holds every SM.
 """
 from __future__ import annotations
 
@@ -27,9 +29,13 @@ from . import binding as B
 
 class LayerGatherSchedule:
     """``layers``: list of (first_tensor, n_tensors) of the plan's tensor list;
-    ``shard_ptrs``: the owners' fp16 shard addresses (one per owner)."""
+    ``shard_ptrs``: the owners' fp16 shard addresses (one per owner);
+    ``engine``: "kernel" (a copy kernel) or "dma" (the copy engines)."""
 
-    def __init__(self, plan: int, layers, shard_ptrs, tensor_sizes, device=None):
+    def __init__(self, plan: int, layers, shard_ptrs, tensor_sizes, device=None, engine: str = "kernel"):
+        if engine not in ("kernel", "dma"):
+            raise ValueError(f"unknown engine {engine!r}")
+        self._gather = B.zero_gather_tensors if engine == "kernel" else B.zero_gather_tensors_dma
         self.plan = plan
         self.layers = list(layers)
         self.shard_ptrs = list(shard_ptrs)
@@ -45,8 +51,8 @@ class LayerGatherSchedule:
         first, count = self.layers[layer]
         cs = self.copy_streams[slot]
         cs.wait_event(free)                           # the slot's last use has finished
-        n = B.zero_gather_tensors(self.plan, first, count, self.shard_ptrs,
-                                  self.buffers[slot].data_ptr(), True, cs.cuda_stream)
+        n = self._gather(self.plan, first, count, self.shard_ptrs, self.buffers[slot].data_ptr(), True,
+                         cs.cuda_stream)
         ready.record(cs)
         self.gathered += n
 
