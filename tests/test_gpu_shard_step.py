@@ -1,8 +1,8 @@
 """The ShardStep object (buffers + C-ABI marshalling around zero_shard_step)
 against the oracle: all owners, a stage-3 owner view with clipping, bf16
-with dynamic loss scaling, and a checkpoint round trip through
-state_dict / load_state_dict that must equal the uninterrupted run bit for
-bit."""
+with dynamic loss scaling, a checkpoint round trip through state_dict /
+load_state_dict, and CUDA-graph replay of captured steps -- the last two
+must equal the uninterrupted direct run bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -162,3 +162,34 @@ def test_checkpoint_round_trip_is_bit_exact(mode):
     ga, wa = B.opt_state_from_bytes(got["opt_state"].numpy().tobytes()), \
         B.opt_state_from_bytes(want["opt_state"].numpy().tobytes())
     assert (ga.t, ga.beta1_pow, ga.beta2_pow, ga.skipped) == (wa.t, wa.beta1_pow, wa.beta2_pow, wa.skipped)
+
+
+@pytest.mark.parametrize("mode", [B.ZERO_MODE_SPECULATIVE, B.ZERO_MODE_STASH], ids=["speculative", "stash"])
+def test_graph_replay_equals_direct_steps(mode):
+    """A step captured as a CUDA graph: each replay advances the device state
+    like a direct call (counter, bias corrections, live slot), so
+    capture-time step + 3 replays equal 4 direct steps bit for bit."""
+    psi, nd, S = 150_001, 4, 1024.0
+    kw = dict(loss_scale=S, weight_decay=0.01, mode=mode, max_grad_norm=0.0 if mode == 0 else 1.0, bucket=40_000)
+    master0 = synth.normal_f32(psi, seed=305, std=0.02)
+    G = _grads(nd, psi, -(-psi // (nd * 256)) * 256 * nd, 0, S)
+    direct = ShardStep(psi, nd, **kw)
+    direct.load_master(torch.from_numpy(master0))
+    _load(direct, G)
+    for _ in range(4):
+        direct.step()
+    want = direct.state_dict()
+    direct.close()
+    g = ShardStep(psi, nd, **kw)
+    g.load_master(torch.from_numpy(master0))
+    _load(g, G)
+    graph = g.capture()                  # runs one step eagerly, then records one
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    got = g.state_dict()
+    assert g.result().t == 4
+    del graph
+    g.close()
+    for k in ("master", "exp_avg", "exp_avg_sq", "params"):
+        assert torch.equal(got[k], want[k]), k

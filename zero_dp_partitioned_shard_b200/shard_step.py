@@ -119,6 +119,21 @@ class ShardStep:
         B.zero_shard_step(self.plan, self.hp, self.args, self._stream())
         return self.result_buf
 
+    def capture(self, steps: int = 1) -> torch.cuda.CUDAGraph:
+        """Records ``steps`` consecutive steps as one CUDA graph; each
+        ``replay()`` then runs them with a single launch.  Everything a step
+        depends on stays in device memory (the step counter, the bias
+        corrections, the live slot, the dynamic loss scale), so a replay is
+        the next steps, not a repeat.  The buffers must not move; refill
+        ``grads`` in stream order between replays."""
+        self.step()                      # resolves launch geometry outside the capture
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(steps):
+                self.step()
+        return graph
+
     def result(self) -> B.StepResult:
         """The last step's result (synchronises with the device)."""
         return B.step_result_from_bytes(self.result_buf.cpu().numpy().tobytes())
