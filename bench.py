@@ -694,7 +694,12 @@ def main():
     if not args.no_e2e:
         import psutil
         need = bench.grad_bytes
-        if psutil.virtual_memory().available > 2.5 * need:
+        # every rank on this node pins its own copy; all ranks must agree on
+        # running the leg, since it holds collectives (barrier, max over ranks)
+        n_local = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+        fits = psutil.virtual_memory().available > 2.5 * need * n_local
+        fits = max_over_ranks(0.0 if fits else 1.0, world) == 0.0
+        if fits:
             g_host = torch.empty(bench.grads.numel(), dtype=bench.grads.dtype, pin_memory=True)
             g_host.copy_(bench.grads)
             r_host = torch.empty(B.RESULT_BYTES, dtype=torch.uint8, pin_memory=True)
@@ -718,7 +723,8 @@ def main():
                    "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps}
             del g_host
         else:
-            e2e = {"value": None, "unit": UNIT, "skipped": "host memory below 2.5x the gradient bytes"}
+            e2e = {"value": None, "unit": UNIT,
+                   "skipped": "host memory below 2.5x the gradient bytes of every rank on the node"}
 
     peak, peak_kind = measured_hbm_peak()
     k_bytes = bench.owned * update_launch_bytes(k_nd, wl["mode"], n_dests)
