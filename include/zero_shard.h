@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 7
+#define ZERO_SHARD_ABI_VERSION 8
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -378,6 +378,20 @@ ZERO_API zero_status zero_workspace_bytes(const zero_plan_t* plan, const zero_hp
 ZERO_API zero_status zero_shard_step(const zero_plan_t* plan, const zero_hparams* hp,
                             const zero_step_args* args, void* stream);
 
+/* Everything zero_shard_step (and its two halves, zero_shard_step_begin and
+ * _end) would do for these arguments except enqueueing work: the same
+ * validation, then each kernel the call would launch is loaded and its
+ * launch geometry (SM count, blocks per SM, shared-memory limit) resolved
+ * and cached for the current device.  Launches nothing, records no timing
+ * event, touches no device memory and changes no optimizer state, so the
+ * next zero_shard_step is the first step.  Call it before capturing steps
+ * into a CUDA graph: the captured calls then neither load a kernel nor query
+ * the device.  Returns the status zero_shard_step would return for these
+ * arguments, minus the launch-time CUDA errors (nothing is launched).  Not a
+ * page's operation: a host-side convenience of this library. */
+ZERO_API zero_status zero_shard_step_prepare(const zero_plan_t* plan, const zero_hparams* hp,
+                                             const zero_step_args* args);
+
 /* ---- split step: one owner per process -------------------------------------- */
 /* When each owner runs in its own process (one GPU each), a step's global
  * decisions -- skip on a non-finite gradient anywhere, the global clip norm --
@@ -427,8 +441,10 @@ ZERO_API zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hpa
  *     ZERO_ERR_WORKSPACE before anything is launched (zero_workspace_bytes
  *     tells the size in advance).
  *   - The first call on a device resolves the array's device address with
- *     that device current and caches it; make that first call before any
- *     stream capture begins.
+ *     that device current and caches it for the current CUDA context; make
+ *     that first call before any stream capture begins.  The address lives
+ *     as long as that context: after cudaDeviceReset (or any teardown of
+ *     the context) the next call, in the new context, resolves it again.
  *   - Every call on a device shares the one array, which keeps the last
  *     call's contents.  Each call rewrites the header and every partial it
  *     reads before reading it, so nothing has to start at zero.  Calls whose
@@ -438,11 +454,12 @@ ZERO_API zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hpa
 ZERO_API zero_status zero_shard_step_static_scratch(const zero_plan_t* plan, const zero_hparams* hp,
                                                     const zero_step_args* args, void* stream);
 
-/* Reduce-scatter with retention (ZeRO stage 2, P_os+g): each gradient is
- * reduced only on the process that owns its partition, which keeps the
- * result, and the full gradients can then be released -- "ZeRO: partitioning
- * training state across GPUs" (upskillscore.com), "How it works";
- * "ZeRO memory optimization" (trishampatil.com), "ZeRO-2".
+/* Reduce-scatter with retention (ZeRO stage 2, P_os+g): the owner of a slice
+ * keeps the rank-order sum of that slice's gradients, after which no rank
+ * needs its full gradient buffer for that slice any more.  Stage 2 as
+ * described in "ZeRO: partitioning training state across GPUs"
+ * (upskillscore.com), "How it works", and "ZeRO memory optimization"
+ * (trishampatil.com), "ZeRO-2".
  *   For the owners owner_first .. owner_first + owner_count - 1 of args and
  *   the flat range of bucket `bucket` of the plan (bucket < 0: the owners'
  *   whole range; a plan without buckets has the one bucket 0), writes

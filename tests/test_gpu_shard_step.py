@@ -166,9 +166,9 @@ def test_checkpoint_round_trip_is_bit_exact(mode):
 
 @pytest.mark.parametrize("mode", [B.ZERO_MODE_SPECULATIVE, B.ZERO_MODE_STASH], ids=["speculative", "stash"])
 def test_graph_replay_equals_direct_steps(mode):
-    """A step captured as a CUDA graph: each replay advances the device state
-    like a direct call (counter, bias corrections, live slot), so
-    capture-time step + 3 replays equal 4 direct steps bit for bit."""
+    """A step captured as a CUDA graph: capturing applies no step, and each
+    replay advances the device state like a direct call (counter, bias
+    corrections, live slot), so 4 replays equal 4 direct steps bit for bit."""
     psi, nd, S = 150_001, 4, 1024.0
     kw = dict(loss_scale=S, weight_decay=0.01, mode=mode, max_grad_norm=0.0 if mode == 0 else 1.0, bucket=40_000)
     master0 = synth.normal_f32(psi, seed=305, std=0.02)
@@ -183,8 +183,17 @@ def test_graph_replay_equals_direct_steps(mode):
     g = ShardStep(psi, nd, **kw)
     g.load_master(torch.from_numpy(master0))
     _load(g, G)
-    graph = g.capture()                  # runs one step eagerly, then records one
-    for _ in range(3):
+    before = g.state_dict()
+    launches = B.zero_launch_count()
+    B.zero_shard_step_prepare(g.plan, g.hp, g.args)
+    assert B.zero_launch_count() == launches          # prepare launches nothing
+    graph = g.capture()                  # prepares again, then records one step
+    torch.cuda.synchronize()
+    assert g.opt().t == 0
+    after = g.state_dict()
+    for k in before:
+        assert torch.equal(after[k], before[k]), f"capture changed {k}"
+    for _ in range(4):
         graph.replay()
     torch.cuda.synchronize()
     got = g.state_dict()

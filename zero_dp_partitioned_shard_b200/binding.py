@@ -139,6 +139,7 @@ SIGNATURES = {
     "zero_workspace_bytes": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), C.POINTER(C.c_size_t)]),
     "zero_shard_step": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_static_scratch": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
+    "zero_shard_step_prepare": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs)]),
     "zero_shard_step_begin": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_shard_step_end": (_S, [_P, C.POINTER(HParams), C.POINTER(StepArgs), _P]),
     "zero_gather_params": (_S, [_P, _P, _P, _P]),
@@ -170,7 +171,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 7:
+        if L.zero_abi_version() != 8:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -257,6 +258,11 @@ def zero_workspace_bytes(plan: int, hp: HParams, args: StepArgs) -> int:
 
 def zero_shard_step(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:
     _check(lib().zero_shard_step(plan, C.byref(hp), C.byref(args), stream), "zero_shard_step")
+
+
+def zero_shard_step_prepare(plan: int, hp: HParams, args: StepArgs) -> None:
+    """Validates a step and loads / sizes its kernels without launching anything."""
+    _check(lib().zero_shard_step_prepare(plan, C.byref(hp), C.byref(args)), "zero_shard_step_prepare")
 
 
 def zero_shard_step_static_scratch(plan: int, hp: HParams, args: StepArgs, stream: int = 0) -> None:

@@ -366,13 +366,16 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
 
     if (spec) {
         if (first_half) {
-            if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+            if (ev0 && !zs::preparing() && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
                 return cuda_fail(e, "timing event");
-            for (const auto& b : lp.buckets)
-                for (const auto& l : b)
-                    if ((e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, peers, str)) != cudaSuccess)
-                        return cuda_fail(e, "update launch");
-            if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+            // Buckets are only the granularity at which gradients become
+            // ready; nothing orders them inside one call, so the update walks
+            // the whole range in as few launches as the segment table allows.
+            for (const auto& l : lp.whole)
+                if (l.count > 0 &&
+                    (e = zs::launch_update(zs::kSrcGradsSpeculative, lp.vec, u, l, peers, str)) != cudaSuccess)
+                    return cuda_fail(e, "update launch");
+            if (ev1 && !zs::preparing() && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
                 return cuda_fail(e, "timing event");
             if (phase == PHASE_BEGIN && (e = zs::launch_vote_local(ws, partials, 0, str)) != cudaSuccess)
                 return cuda_fail(e, "vote launch");
@@ -420,12 +423,12 @@ static zero_status run_step(const zero_plan_t* plan, const zero_hparams* hp, con
             (e = zs::launch_vote_apply(ws, false, h.max_grad_norm, st, res, str)) != cudaSuccess)
             return cuda_fail(e, "vote launch");
         const int src = h.mode == ZERO_MODE_STASH ? zs::kSrcStash : zs::kSrcGradsInPlace;
-        if (ev0 && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
+        if (ev0 && !zs::preparing() && (e = cudaEventRecord(ev0, str)) != cudaSuccess)
             return cuda_fail(e, "timing event");
         for (const auto& l : lp.whole)
             if (l.count > 0 && (e = zs::launch_update(src, lp.vec, u, l, peers, str)) != cudaSuccess)
                 return cuda_fail(e, "update launch");
-        if (ev1 && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
+        if (ev1 && !zs::preparing() && (e = cudaEventRecord(ev1, str)) != cudaSuccess)
             return cuda_fail(e, "timing event");
     }
     return ZERO_OK;
@@ -495,6 +498,20 @@ zero_status zero_shard_step_end(const zero_plan_t* plan, const zero_hparams* hp,
                                 const zero_step_args* args, void* stream)
 {
     return run_step(plan, hp, args, stream, PHASE_END);
+}
+
+zero_status zero_shard_step_prepare(const zero_plan_t* plan, const zero_hparams* hp,
+                                    const zero_step_args* args)
+{
+    // the host logic of a whole step and of its two halves, each launch
+    // replaced by loading its kernel (the geometry is cached on the way)
+    zs::PrepareScope scope;
+    zero_status s = run_step(plan, hp, args, nullptr, PHASE_ALL);
+    if (s == ZERO_OK)
+        s = run_step(plan, hp, args, nullptr, PHASE_BEGIN);
+    if (s == ZERO_OK)
+        s = run_step(plan, hp, args, nullptr, PHASE_END);
+    return s;
 }
 
 // Launches copies of shard pieces, at most kMaxSegs per launch; compact

@@ -1172,13 +1172,21 @@ static int64_t seg_work(const SegList& s, bool vec)
 // launchers
 // ---------------------------------------------------------------------------
 
-// Launch with programmatic stream serialization: the kernel may begin while
-// its predecessor in the stream drains (it orders itself with
-// griddepcontrol.wait).  Used for the kernels after the first of a step.
+// Every kernel launch of the library goes through here.  overlapped: with
+// programmatic stream serialization, so the kernel may begin while its
+// predecessor in the stream drains (it orders itself with
+// griddepcontrol.wait); used for the kernels after the first of a step.
+// While a prepare call is running (zs::preparing()) the kernel is only
+// loaded -- the caller has already resolved its geometry -- and nothing is
+// enqueued or counted.
 template <typename... Params, typename... Args>
-static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
-                                     cudaStream_t s, Args... args)
+static cudaError_t launch_k(bool overlapped, void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                            cudaStream_t s, Args... args)
 {
+    if (preparing()) {
+        cudaFuncAttributes fa;
+        return cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
@@ -1188,24 +1196,37 @@ static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, u
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+    cfg.numAttrs = overlapped ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
+}
+
+template <typename... Params, typename... Args>
+static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                                     cudaStream_t s, Args... args)
+{
+    return launch_k(true, kernel, grid, block, smem, s, args...);
+}
+
+template <typename... Params, typename... Args>
+static cudaError_t launch_plain(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                                cudaStream_t s, Args... args)
+{
+    return launch_k(false, kernel, grid, block, smem, s, args...);
 }
 
 cudaError_t launch_opt_init(zero_opt_state* st, float scale, float growth, float backoff, int32_t interval,
                             cudaStream_t s)
 {
-    zs_opt_init_kernel<<<1, 1, 0, s>>>(st, scale, growth, backoff, interval);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(zs_opt_init_kernel, 1, 1, 0, s, st, scale, growth, backoff, interval);
 }
 
 cudaError_t launch_prep(const zero_opt_state* st, WsHeader* ws, float beta1, float beta2, float static_inv,
                         double scale_mult, cudaStream_t s)
 {
-    zs_prep_kernel<<<1, 1, 0, s>>>(st, ws, beta1, beta2, static_inv, scale_mult);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(zs_prep_kernel, 1, 1, 0, s, st, ws, beta1, beta2, static_inv, scale_mult);
 }
 
 // The peer table as the kernel parameter of a PEER / non-PEER instantiation.
@@ -1226,9 +1247,7 @@ static cudaError_t launch_update_t(const UpdateArgs& a, const SegList& segs, con
     cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, peer_param<PEER>(peers));
-    count_launches(1);
-    return e;
+    return launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, peer_param<PEER>(peers));
 }
 
 template <int SRC, bool BF>
@@ -1311,10 +1330,8 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
     int64_t grid = (int64_t)sms * ps.ctas_per_sm;
     grid = tiles < grid ? tiles : grid;
     grid = grid < 1 ? 1 : grid;
-    e = launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages,
-                          peer_param<PEER>(peers));
-    count_launches(1);
-    return e;
+    return launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages,
+                             peer_param<PEER>(peers));
 }
 
 template <int SRC, bool BF, bool PEER>
@@ -1380,10 +1397,8 @@ int stats_blocks(bool vec, const SegList& segs)
 template <bool VEC, bool STASH, bool BF, bool PEER>
 static cudaError_t launch_stats_t(const StatsArgs& a, const SegList& segs, const PeerTable* peers, cudaStream_t s)
 {
-    const cudaError_t e = launch_overlapped(zs_stats_kernel<VEC, STASH, BF, PEER>, stats_blocks(VEC, segs),
-                                            kThreads, 0, s, a, segs, peer_param<PEER>(peers));
-    count_launches(1);
-    return e;
+    return launch_overlapped(zs_stats_kernel<VEC, STASH, BF, PEER>, stats_blocks(VEC, segs), kThreads, 0, s, a,
+                             segs, peer_param<PEER>(peers));
 }
 
 template <bool BF, bool PEER>
@@ -1410,26 +1425,19 @@ cudaError_t launch_stats(bool vec, const StatsArgs& a, const SegList& segs, cons
 cudaError_t launch_finalize(WsHeader* ws, const double* partials, int64_t n, float max_norm,
                             zero_opt_state* st, zero_step_result* res, cudaStream_t s)
 {
-    const cudaError_t e = launch_overlapped(zs_finalize_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n,
-                                            max_norm, st, res);
-    count_launches(1);
-    return e;
+    return launch_overlapped(zs_finalize_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n, max_norm, st, res);
 }
 
 cudaError_t launch_vote_local(WsHeader* ws, const double* partials, int64_t n, cudaStream_t s)
 {
-    const cudaError_t e = launch_overlapped(zs_vote_local_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n);
-    count_launches(1);
-    return e;
+    return launch_overlapped(zs_vote_local_kernel, 1, kFinalizeThreads, 0, s, ws, partials, n);
 }
 
 cudaError_t launch_vote_apply(WsHeader* ws, bool speculative, float max_norm, zero_opt_state* st,
                               zero_step_result* res, cudaStream_t s)
 {
     // an ordinary launch: the caller's all-reduce of the vote comes before it
-    zs_vote_apply_kernel<<<1, 1, 0, s>>>(ws, speculative ? 1 : 0, max_norm, st, res);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(zs_vote_apply_kernel, 1, 1, 0, s, ws, speculative ? 1 : 0, max_norm, st, res);
 }
 
 template <bool VEC, bool BF, bool PEER>
@@ -1441,10 +1449,8 @@ static cudaError_t launch_commit_t(const UpdateArgs& a, const SegList& segs, boo
     cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    e = launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res,
-                          peer_param<PEER>(peers));
-    count_launches(1);
-    return e;
+    return launch_overlapped(kernel, blocks, kThreads, 0, s, a, segs, bookkeeping ? 1 : 0, st, res,
+                             peer_param<PEER>(peers));
 }
 
 template <bool BF, bool PEER>
@@ -1474,9 +1480,7 @@ static cudaError_t launch_reduce_t(const uint16_t* grads, uint16_t* out, int nd,
     cudaError_t e = grid_for(kernel, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    kernel<<<blocks, kThreads, 0, s>>>(grads, out, nd, segs, peer_param<PEER>(peers));
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(kernel, blocks, kThreads, 0, s, grads, out, nd, segs, peer_param<PEER>(peers));
 }
 
 template <bool BF, bool PEER>
@@ -1504,9 +1508,7 @@ static cudaError_t launch_cast_t(const float* master, uint16_t* params, const Se
     cudaError_t e = grid_for(zs_cast_kernel<VEC, BF>, seg_work(segs, VEC), 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    zs_cast_kernel<VEC, BF><<<blocks, kThreads, 0, s>>>(master, params, segs);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(zs_cast_kernel<VEC, BF>, blocks, kThreads, 0, s, master, params, segs);
 }
 
 cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* params, const SegList& segs,
@@ -1527,9 +1529,7 @@ cudaError_t launch_gather(uint16_t* dst, const GatherList& g, bool streaming_sto
     cudaError_t e = grid_for(kernel, w, 0, &blocks);
     if (e != cudaSuccess)
         return e;
-    kernel<<<blocks, kThreads, 0, s>>>(dst, g);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_plain(kernel, blocks, kThreads, 0, s, dst, g);
 }
 
 } // namespace zs

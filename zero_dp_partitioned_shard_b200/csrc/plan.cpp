@@ -34,6 +34,11 @@ void clear_error() { g_last_error[0] = '\0'; }
 
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+static thread_local bool t_preparing = false;
+bool preparing() { return t_preparing; }
+PrepareScope::PrepareScope() { t_preparing = true; }
+PrepareScope::~PrepareScope() { t_preparing = false; }
+
 } // namespace zs
 
 using zs::fail;

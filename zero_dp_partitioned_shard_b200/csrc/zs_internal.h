@@ -31,6 +31,15 @@ void clear_error();
 void count_launches(uint64_t n);
 long long wait_budget_cycles();  // current budget of a bounded pipeline wait
 
+// A prepare call (zero_shard_step_prepare) runs the step's host logic with
+// every launch replaced by loading the kernel: launch geometry is resolved
+// and cached, nothing is enqueued.  Per calling thread.
+bool preparing();
+struct PrepareScope {
+    PrepareScope();
+    ~PrepareScope();
+};
+
 // ---- launch geometry ------------------------------------------------------------
 constexpr int kThreads = 256;          // threads per block of the streaming kernels
 constexpr int kMaxSegs = 64;           // segments per launch (kernel parameter table)

@@ -121,13 +121,15 @@ class ShardStep:
 
     def capture(self, steps: int = 1) -> torch.cuda.CUDAGraph:
         """Records ``steps`` consecutive steps as one CUDA graph; each
-        ``replay()`` then runs them with a single launch.  Everything a step
+        ``replay()`` then runs them with a single launch.  Capturing applies
+        no step: the first replay is the next step.  Everything a step
         depends on stays in device memory (the step counter, the bias
-        corrections, the live slot, the dynamic loss scale), so a replay is
-        the next steps, not a repeat.  The buffers must not move; refill
-        ``grads`` in stream order between replays."""
-        self.step()                      # resolves launch geometry outside the capture
-        torch.cuda.synchronize(self.device)
+        corrections, the live slot, the dynamic loss scale), so each replay
+        continues from the last one rather than repeating it.  The buffers
+        must not move; refill ``grads`` in stream order between replays."""
+        # load the step's kernels and size their grids before the capture
+        # opens; this launches nothing and leaves the state untouched
+        B.zero_shard_step_prepare(self.plan, self.hp, self.args)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             for _ in range(steps):
