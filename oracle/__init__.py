@@ -103,7 +103,7 @@ def lib():
                                       C.POINTER(HParams), C.POINTER(OptState),
                                       _I32, C.c_float, C.c_int, C.POINTER(StepInfo)]),
             "oracle_grad_sumsq": (C.c_double, [_P, _I64, _I32, _I64, C.POINTER(HParams),
-                                               C.c_double, C.POINTER(_I32)]),
+                                               _P, C.POINTER(_I32)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -388,13 +388,20 @@ def update_elements(G: np.ndarray, master: np.ndarray, exp_avg: np.ndarray,
                                  float(clip_coef), float(bc1), float(bc2), threads)
 
 
-def grad_sumsq(G: np.ndarray, hp: HP, acc: float = 0.0) -> tuple[float, bool]:
-    """Streamed fp64 sum of squares of the unscaled reduced gradient of G [nd, n]."""
+def grad_sumsq(G: np.ndarray, hp: HP, acc: np.ndarray | None = None) -> tuple[float, bool]:
+    """Compensated fp64 sum of squares of the unscaled reduced gradient of G
+    [nd, n].  acc: optional float64[2] Neumaier accumulator {sum,
+    compensation}, updated in place, to stream a problem through in pieces:
+    one acc carried along gives the single-pass sum bit for bit; separate
+    accs per piece add up exactly with math.fsum over all their terms."""
     G = np.ascontiguousarray(G, dtype=np.uint16)
+    if acc is None:
+        acc = np.zeros(2, np.float64)
+    assert acc.dtype == np.float64 and acc.shape == (2,) and acc.flags["C_CONTIGUOUS"]
     h = hp._c()
     bad = _I32(0)
     s = lib().oracle_grad_sumsq(_ptr(G), G.shape[1], G.shape[0], G.shape[1], C.byref(h),
-                                float(acc), C.byref(bad))
+                                _ptr(acc), C.byref(bad))
     return s, bool(bad.value)
 
 

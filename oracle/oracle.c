@@ -744,19 +744,26 @@ int oracle_step(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t psi,
 }
 
 /* Sum of squares of the unscaled reduced gradient over n elements (the same
- * compensated fp64 sum as oracle_step), added to acc.  Lets a caller stream a
- * large problem through in pieces.  *nonfinite is set to 1 if any reduced
- * element is non-finite. */
+ * compensated fp64 sum as oracle_step), added into the Neumaier accumulator
+ * acc = {running sum, compensation}, which is updated in place and may carry
+ * over from earlier pieces.  A caller that streams a large problem through in
+ * pieces and passes the same acc along gets exactly the single-pass sum (the
+ * same additions in the same order); pieces summed with separate accumulators
+ * stay exact when their sum and compensation terms are added exactly (for
+ * instance with Python's math.fsum).  Returns acc[0] + acc[1].  *nonfinite is
+ * set to 1 if any reduced element is non-finite. */
 double oracle_grad_sumsq(const uint16_t* G, int64_t rank_stride, int32_t nd, int64_t n,
-                         const oracle_hparams* hp, double acc, int32_t* nonfinite)
+                         const oracle_hparams* hp, double acc[2], int32_t* nonfinite)
 {
     const float inv = unscale_factor(hp, nd);
-    comp_sum a = {acc, 0.0};
+    comp_sum a = {acc[0], acc[1]};
     for (int64_t i = 0; i < n; ++i) {
         float g = rank_sum_of(G, rank_stride, nd, i, hp->storage) * inv;
         if (!isfinite(g))
             *nonfinite = 1;
         comp_add(&a, (double)g * (double)g);
     }
+    acc[0] = a.s;
+    acc[1] = a.c;
     return a.s + a.c;
 }

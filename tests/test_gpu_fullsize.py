@@ -252,7 +252,8 @@ def test_7p5b_gather_assembly_sampled_windows():
 
 def _streamed_oracle_norm(bn, hp, chunk=1 << 24):
     """Oracle fp64 sum of squares over all owned elements, chunk by chunk from
-    the device bytes (chunks summed in order; within a chunk left to right)."""
+    the device bytes: each chunk's compensated sum keeps its compensation term,
+    and all the chunks' terms are added exactly (math.fsum)."""
     starts = list(range(0, bn.owned, chunk))
     workers = oracle.host_threads()
     parts = []
@@ -262,16 +263,17 @@ def _streamed_oracle_norm(bn, hp, chunk=1 << 24):
         G = torch.stack([bn.grads[r * bn.stride + s:r * bn.stride + e] for r in range(bn.nd)])
         return G.view(torch.int16).cpu().numpy().view(np.uint16)
 
+    def chunk_sumsq(G):
+        acc = np.zeros(2, np.float64)
+        _, bad = oracle.grad_sumsq(G, hp, acc)
+        return acc, bad
+
     with cf.ThreadPoolExecutor(max_workers=workers) as ex:
         for w in range(0, len(starts), workers):   # bounded host memory: one wave at a time
             wave = [load(s) for s in starts[w:w + workers]]
-            parts += list(ex.map(lambda G: oracle.grad_sumsq(G, hp), wave))
-    total = 0.0
-    bad = False
-    for s, b in parts:
-        total += s
-        bad |= b
-    return math.sqrt(total), bad
+            parts += list(ex.map(chunk_sumsq, wave))
+    total = math.fsum(x for acc, _ in parts for x in acc)
+    return math.sqrt(total), any(b for _, b in parts)
 
 
 def test_24l_d2048_nd16_bucketed_clip_stash_sampled_with_injection():
@@ -327,5 +329,29 @@ def test_sweep_points_full_parity(psi, nd, stage):
                 stage=stage)
     o = run_oracle(pb, to_oracle_hp(hp), threads=oracle.host_threads())
     assert_f32_close(g.master, o.master, 2, "master")
+    assert_f32_close(g.exp_avg, o.exp_avg, 2, "exp_avg")
     assert_f32_close(g.exp_avg_sq, o.exp_avg_sq, 2, "exp_avg_sq")
     assert_f16_close(g.params, o.params, 1, "params")
+    assert [r.overflow for r in g.results] == [i["overflow"] for i in o.infos] == [0]
+    assert g.opt.t == o.opt.t == 1 and g.results[-1].t == 1
+
+
+@pytest.mark.parametrize("psi,nd,stage", [
+    (256 << 20, 1, 1),      # Nd <= 2: the low-byte streams
+    (256 << 20, 2, 2),      # ... in 8 buckets
+    (1 << 30, 64, 3),       # one owner of 64 at 1B (the one-owner view)
+])
+def test_sweep_points_large_sampled(psi, nd, stage):
+    """The sweep's large points in the configuration the sweep times: every
+    owned element is updated on the GPU, sampled elements (random plus every
+    shard, bucket and vector boundary) are recomputed by the oracle from the
+    device bytes over two steps."""
+    free, _ = torch.cuda.mem_get_info()
+    wl = bench.sweep_workload(psi, nd, stage, free)
+    assert (wl["owner_count"] == 1) == (nd == 64)
+    bn = bench.Bench(wl, None, seed=11 + nd)
+    try:
+        res = _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=nd + stage)
+        assert [r.overflow for r in res] == [0, 0] and res[-1].t == 2
+    finally:
+        bn.close()

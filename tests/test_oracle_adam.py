@@ -164,6 +164,30 @@ def test_norm_is_the_exact_sum_of_squares():
     assert infos[0]["grad_norm"] == math.sqrt(infos[0]["sumsq"])
 
 
+def test_streamed_sum_of_squares_carries_its_compensation():
+    """Pieces streamed with one carried accumulator give the single-pass sum
+    bit for bit; pieces with their own accumulators, added exactly
+    (math.fsum of every sum and compensation term), stay within 2 ulp of the
+    exactly rounded sum of the exact squares."""
+    nd, n, S = 3, 300_007, 64.0
+    G = synth.grads_f16(nd, n, seed=33, std=1e-2, scale=S)
+    G[:, ::613] = np.float16(3000.0).view(np.uint16)
+    hp = oracle.HP(loss_scale=S)
+    whole, _ = oracle.grad_sumsq(G, hp)
+    cuts = [0, 1, 4097, 100_000, 100_001, 250_000, n]
+    carried = np.zeros(2, np.float64)
+    separate = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        oracle.grad_sumsq(np.ascontiguousarray(G[:, a:b]), hp, carried)
+        own = np.zeros(2, np.float64)
+        oracle.grad_sumsq(np.ascontiguousarray(G[:, a:b]), hp, own)
+        separate += own.tolist()
+    assert carried.sum() == whole and carried[0] + carried[1] == whole
+    g = oracle.all_reduce(G, n) * np.float32(1.0 / S)
+    exact = math.fsum((g.astype(np.float64) ** 2).tolist())
+    assert abs(math.fsum(separate) - exact) <= 2 * math.ulp(exact)
+
+
 def test_average_over_nd_divides_by_nd():
     nd, n, S = 8, 64, 1024.0
     G, g = _const_grads(np.full(n, 2.0 ** -8), nd, S)
