@@ -55,8 +55,8 @@ def test_tiny_workload_bf16(mode, stage):
     assert g.opt.t == 3
 
 
-# (psi, nd, align, bucket): Nd 1 and 2 and the stash mode take the bulk-copy
-# pipeline; the others the register path; align 1 the scalar path
+# (psi, nd, align, bucket): vectorised Nd <= 16 and the stash mode take the
+# bulk-copy pipeline; Nd = 64 the register path; align 1 the scalar path
 RAGGED = [(1, 1, 1, 0), (7, 3, 1, 0), (4097, 2, 8, 1000), (100_003, 1, 256, 0), (100_003, 7, 16, 4096),
           (200_001, 64, 256, 8192), (65_539, 2, 1, 0)]
 

@@ -2,7 +2,12 @@
 //
 // The step is HBM-bound streaming work (about 20 fp32 operations, one square
 // root and three divisions per parameter against 2*Nd + 26 bytes), so it uses
-// no tensor cores.  Design points for B200:
+// no tensor cores.  The update runs as a bulk-copy pipeline (warp-specialised:
+// one producer warp streams tiles into a shared-memory ring with
+// cp.async.bulk, eight consumer warps compute from it) for up to 16
+// contributions and for the stash, and on the register path below for more.
+// Design points of the register path, which the statistics, reduce, commit
+// and cast kernels share:
 //   * one thread owns 8 consecutive parameters per iteration: every access is
 //     a 16-byte vector (fp16 x8 or fp32 x4) and a warp touches 512 contiguous
 //     bytes of each stream; loads bypass L1 and are marked evict-first, since
@@ -189,19 +194,23 @@ __device__ __forceinline__ void store_param1(uint16_t* params, const PeerParam<P
 }
 
 // Rank-order sum of the Nd contributions of 8 consecutive parameters: the
-// loads of each group of 8 ranks are issued together, then added in order.
-template <bool BF, class Ranks>
+// loads of the first G ranks are issued together, then those of each further
+// group of 8, and every group is added in rank order.  G = 8 suits the update
+// kernel, which also holds master/m/v in registers; the statistics pass has
+// the registers to keep all 16 contributions of a 16-rank step in flight
+// (measured 1.00 of the copy bandwidth against 0.94-0.97 with G = 8).
+template <bool BF, int G = 8, class Ranks>
 __device__ __forceinline__ void rank_sum8(const Ranks& rk, int nd, float s[8])
 {
     {
-        uint4 x[8];
+        uint4 x[G];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < G; ++u)
             if (u < nd)
                 x[u] = ld_stream(rk.at(u));
         unpack_h8<BF>(x[0], s);
 #pragma unroll
-        for (int u = 1; u < 8; ++u) {
+        for (int u = 1; u < G; ++u) {
             if (u < nd) {
                 float f[8];
                 unpack_h8<BF>(x[u], f);
@@ -211,7 +220,7 @@ __device__ __forceinline__ void rank_sum8(const Ranks& rk, int nd, float s[8])
             }
         }
     }
-    for (int r = 8; r < nd; r += 8) {
+    for (int r = G; r < nd; r += 8) {
         uint4 x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
@@ -818,7 +827,7 @@ zs_stats_kernel(const StatsArgs a, const __grid_constant__ SegList segs, const _
         segs,
         [&](const Seg& sg, int64_t e) {
             float g[8];
-            rank_sum8<BF>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd, g);
+            rank_sum8<BF, 16>(ranks_at<PEER>(a.grads, pt, sg, e), a.nd, g);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 g[q] = __fmul_rn(g[q], inv);
@@ -1270,34 +1279,50 @@ static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegLi
 }
 
 // Shape of the pipelined update for a given source: elements per consumer
-// thread (tile = 256 x EPT), ring stages and CTAs per SM.  A stage holds one
-// tile of master/m/v plus the tile's source bytes; it is kept <= 48 KB for
-// EPT > 1, and two CTAs share an SM when three or more stages fit in half of
-// its shared memory.
+// thread (tile = 256 x EPT), ring stages and CTAs per SM.  Chosen by
+// measurement on one B200 (1B-parameter streams, 30- and 200-launch runs,
+// the latter with the SM clock held near 1.5 GHz by the power cap), every
+// shape bit-identical to the register path:
+//   * contributions, Nd <= 8: EPT 4, 2 stages, 3 CTAs per SM -- 0.92 (Nd 1),
+//     0.93 (2), 0.97 (4), 1.00 (8) of the copy bandwidth, against 0.79-0.95
+//     for the register path and 0.90-1.00 for deeper 2-CTA rings;
+//   * contributions, Nd <= 16: EPT 4, 2 stages, 2 CTAs (3 no longer fit):
+//     1.02 at Nd = 16 against 0.94-0.97 for the register path;
+//   * the 4-byte stash: EPT 8, 2 stages, 2 CTAs -- 0.96 against 0.89 for a
+//     3-stage ring and 0.92 for the register path.
+// A shallow ring with more CTAs per SM beat every deeper one: the same bytes
+// in flight per SM, spread over more independent producers.  Beyond Nd = 16
+// a tile needs Nd + 3 small copies and the copy issue, not HBM, limits the
+// pipeline (0.6 at Nd = 32 and 64); the register path takes those.
 struct PipeShape {
     int ept = 0, stages = 0, ctas_per_sm = 0, smem = 0;
 };
 
+constexpr int kPipeMaxNd = 16;
+
 static bool pipe_shape(int src, int nd, PipeShape* ps)
 {
-    const int e = 12 + (src == kSrcStash ? 4 : 2 * nd);
-    const int ept = 2048 * e <= 32 * 1024 ? 8
-                  : (1024 * e <= 48 * 1024 ? 4 : (512 * e <= 48 * 1024 ? 2 : (256 * e <= 72 * 1024 ? 1 : 0)));
-    if (!ept)
+    const bool stash = src == kSrcStash;
+    if (!stash && nd > kPipeMaxNd)
         return false;
-    const int stage = kPipeConsumers * ept * e;
-    int ctas = 2, stages = (110 * 1024 - kPipeHeaderBytes) / stage;
-    if (stages < 3) {
-        ctas = 1;
-        stages = (220 * 1024 - kPipeHeaderBytes) / stage;
+    const int e = 12 + (stash ? 4 : 2 * nd); // bytes per element of one stage
+    PipeShape p;
+    if (stash) {
+        p.ept = 8, p.stages = 2, p.ctas_per_sm = 2;
+    } else {
+        p.ept = 4, p.stages = 2, p.ctas_per_sm = 3;
     }
-    stages = stages > 8 ? 8 : stages;
-    if (stages < 2)
+    // CTAs per SM that the shared memory allows (228 KB per SM, 1 KB of it
+    // reserved per CTA); the launch also checks the occupancy it gets
+    for (;;) {
+        p.smem = kPipeHeaderBytes + p.stages * kPipeConsumers * p.ept * e;
+        if (p.ctas_per_sm * (p.smem + 1024) <= 228 * 1024 || p.ctas_per_sm == 1)
+            break;
+        --p.ctas_per_sm;
+    }
+    if (p.smem > 220 * 1024 + kPipeHeaderBytes)
         return false;
-    ps->ept = ept;
-    ps->stages = stages;
-    ps->ctas_per_sm = ctas;
-    ps->smem = kPipeHeaderBytes + stages * stage;
+    *ps = p;
     return true;
 }
 
@@ -1323,11 +1348,28 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
             g_smem_set[key] = 220 * 1024 + kPipeHeaderBytes;
         }
     }
+    int occ = 0;
+    {
+        const std::pair<const void*, int> okey(reinterpret_cast<const void*>(kernel), dev * 4096 + ps.smem / 256);
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_occ.find(okey);
+        if (it != g_occ.end())
+            occ = it->second;
+    }
+    if (occ == 0) {
+        // blocks per SM that fit at this shape (registers, threads, shared memory)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kPipeThreads, ps.smem);
+        if (e != cudaSuccess)
+            return e;
+        occ = occ < 1 ? 1 : occ;
+        std::lock_guard<std::mutex> lk(g_mu);
+        g_occ[std::pair<const void*, int>(reinterpret_cast<const void*>(kernel), dev * 4096 + ps.smem / 256)] = occ;
+    }
     int64_t tiles = 0;
     const int T = kPipeConsumers * EPT;
     for (int i = 0; i < segs.count; ++i)
         tiles += ((segs.seg[i].n >> 3) * 8 + T - 1) / T;
-    int64_t grid = (int64_t)sms * ps.ctas_per_sm;
+    int64_t grid = (int64_t)sms * (ps.ctas_per_sm < occ ? ps.ctas_per_sm : occ);
     grid = tiles < grid ? tiles : grid;
     grid = grid < 1 ? 1 : grid;
     return launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages,
@@ -1338,12 +1380,9 @@ template <int SRC, bool BF, bool PEER>
 static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                  const PeerTable* peers, cudaStream_t s)
 {
-    switch (ps.ept) {
-    case 8: return launch_pipe_t<SRC, 8, BF, PEER>(a, segs, ps, peers, s);
-    case 4: return launch_pipe_t<SRC, 4, BF, PEER>(a, segs, ps, peers, s);
-    case 2: return launch_pipe_t<SRC, 2, BF, PEER>(a, segs, ps, peers, s);
-    default: return launch_pipe_t<SRC, 1, BF, PEER>(a, segs, ps, peers, s);
-    }
+    // pipe_shape chooses 8 (the stash) or 4 (contributions) elements per thread
+    return ps.ept == 8 ? launch_pipe_t<SRC, 8, BF, PEER>(a, segs, ps, peers, s)
+                       : launch_pipe_t<SRC, 4, BF, PEER>(a, segs, ps, peers, s);
 }
 
 // With peer tables the pipeline runs only from the stash (its rank loads stay
@@ -1361,12 +1400,10 @@ static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const P
                   : launch_pipe_f<SRC, false, false>(a, segs, ps, nullptr, s);
 }
 
-// The bulk-copy pipeline pays off where a parameter carries few bytes (the
-// stash source, Nd <= 2: measured 0.87-0.88 of the copy bandwidth against
-// 0.85-0.86 for the register path); from Nd = 4 up the register path, whose
-// groups of 8 rank loads keep more bytes in flight per thread, is faster
-// (0.95-1.02 against 0.64-0.95).
-static bool use_pipeline(int src, int nd) { return src == kSrcStash || nd <= 2; }
+// The bulk-copy pipeline takes the stash source and up to 16 contributions
+// (see pipe_shape for the measurements); the register path, whose groups of
+// 8 rank loads need no copy per rank, takes larger Nd.
+static bool use_pipeline(int src, int nd) { return src == kSrcStash || nd <= kPipeMaxNd; }
 
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
                           cudaStream_t s)
