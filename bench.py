@@ -12,7 +12,8 @@ all-gathered parameter buffer.
 Prints one JSON line (rank 0).  ``value`` is owned parameters updated per
 second over all ranks with inputs resident in HBM; ``e2e`` repeats the
 measurement through the C-ABI call with the step's gradients copied from
-pinned host memory every step and the step result read back; ``roofline``
+pinned host memory every step and the step's product (the updated 16-bit
+parameters) and its result struct copied back; ``roofline``
 reports the update kernel's algorithmic bytes per launch over its CUDA-event
 duration against the measured HBM copy bandwidth; ``cpu_baseline`` times the
 CPU oracle on a bounded sample on this host.
@@ -47,6 +48,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -95,6 +97,15 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     alg = 2 * nd + 26  # Nd fp16 reads, master/m/v read+write (24), fp16 write (2)
     moved = {0: alg, 1: 4 * nd + 26, 2: 2 * nd + 34}[mode]
     return alg, moved
+
+
+def update_kernel_name(nd: int, mode: int, peer: bool = False) -> str:
+    """The library's update kernel for this source: the bulk-copy pipeline for
+    the stash and up to 16 local contributions, the register path otherwise
+    (larger Nd, or contributions read through peer tables)."""
+    if mode == 2 or (nd <= 16 and not peer):
+        return "zs_update_pipe_kernel"
+    return "zs_update_kernel"
 
 
 def update_launch_bytes(nd: int, mode: int, dests: int = 0) -> int:
@@ -320,6 +331,61 @@ class Bench:
         self.B.zero_plan_destroy(self.plan)
 
 
+def timed_steps(bench, steps: int, warmup: int, world: int, local: int, n_ev: int = 2,
+                inject: dict | None = None) -> dict:
+    """Warm-up, then ``steps`` steps timed on the device: CUDA events around the
+    whole region (bracketed by a barrier and a synchronize on both sides) and
+    around each step's update launches; SM clocks sampled during the region.
+    inject: {step: (rank, flat index, value)} -- the value is planted in that
+    rank's gradient before the step and the old value put back after it (a
+    seeded overflow schedule: the step must be skipped).  Returns the region's
+    ms, the per-step update-kernel ms of the applied steps, the skipped count,
+    the library's launches and the clocks."""
+    import torch
+    from zero_dp_partitioned_shard_b200 import binding as B
+    for _ in range(warmup):
+        bench.step()
+    k_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(n_ev)) for _ in range(steps)]
+    for evs in k_events:    # create the CUDA events before handing their handles over
+        for ev in evs:
+            ev.record()
+    inject = inject or {}
+    if inject and bench.wl["layout"] != 0:
+        raise ValueError("the injection schedule addresses the full per-rank gradient layout")
+    planted = {}
+    for k, (rank, i, val) in inject.items():
+        if k < steps:
+            flat = rank * bench.stride + i
+            planted[k] = (flat, bench.grads[flat:flat + 1].clone(), val)
+    skipped0 = B.opt_state_from_bytes(bench.opt_state.cpu().numpy().tobytes()).skipped
+    torch.cuda.synchronize()
+    _barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = B.zero_launch_count()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for k in range(steps):
+        hit = planted.get(k)
+        if hit is not None:
+            bench.grads[hit[0]] = hit[2]
+        bench.step(k_events[k])
+        if hit is not None:
+            bench.grads[hit[0]:hit[0] + 1].copy_(hit[1])
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = B.zero_launch_count() - launches0
+    clk = clocks.stop()
+    _barrier(world)
+    skipped = B.opt_state_from_bytes(bench.opt_state.cpu().numpy().tobytes()).skipped - skipped0
+    return {"ms_total": t_start.elapsed_time(t_end), "launches": launches, "clocks": clk,
+            "skipped": skipped, "injected": len(planted),
+            "kernel_ms": [ev[0].elapsed_time(ev[1]) for k, ev in enumerate(k_events) if k not in planted],
+            "reduce_ms": [ev[2].elapsed_time(ev[3]) for ev in k_events] if n_ev > 2 else []}
+
+
 def _dist():
     import torch
     import torch.distributed as dist
@@ -432,6 +498,95 @@ def run_reference(args, wl_name: str, wl: dict):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def step_alg_bytes(owned: int, assembled: int, nd: int, steps: int, skipped: int) -> int:
+    """Algorithmic bytes of ``steps`` steps of which ``skipped`` were skipped on
+    overflow: an applied step moves (2 Nd + 26) B per owned parameter plus 4 B
+    per assembled one; a skipped step has still read every contribution
+    (2 Nd B per owned parameter) and updates nothing."""
+    return (steps - skipped) * (owned * (2 * nd + 26) + 4 * assembled) + skipped * owned * 2 * nd
+
+
+def config_entry(name: str, wl: dict, args, world: int, local: int, peak: float, seed: int,
+                 inject_rate: float = 0.0, min_ms: float = 400.0) -> dict:
+    """One more workload measured in the same run as the headline: its step
+    time, its update kernel's CUDA-event time against the kernel's own
+    algorithmic bytes, and the whole step's fraction by the workload's
+    algorithmic bytes (assembly included).  The timed steps are at least
+    ``args.steps`` and enough for about ``min_ms`` of device time, so the clock
+    sampler sees the region.  inject_rate > 0 plants a seeded overflow
+    schedule (that share of steps, the first timed step always) in the timed
+    region; skipped steps move only their gradient reads."""
+    import torch
+    from zero_dp_partitioned_shard_b200 import synth
+    torch.cuda.empty_cache()
+    bn = Bench(wl, None, seed=seed)
+    try:
+        for _ in range(args.warmup):
+            bn.step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        bn.step()
+        b.record()
+        torch.cuda.synchronize()
+        one = max(a.elapsed_time(b), 1e-3)
+        steps = max(args.steps, int(math.ceil(min_ms / one)))
+        steps = int(max_over_ranks(float(steps), world))
+        inject = None
+        if inject_rate > 0:
+            inject = synth.inject_schedule(steps, inject_rate, seed=seed * 7 + 1, nd=bn.nd, psi=bn.psi,
+                                           force_step=0)
+        tr = timed_steps(bn, steps, 3, world, local, inject=inject)
+        ms_max = max_over_ranks(tr["ms_total"], world)
+        k_ms = max_over_ranks(statistics.mean(tr["kernel_ms"]), world)
+        nd, mode = wl["nd"], wl["mode"]
+        alg, moved = bytes_per_param(nd, mode)
+        k_bytes = bn.owned * update_launch_bytes(nd, mode)
+        step_bytes = step_alg_bytes(bn.owned, bn.assembled, nd, steps, tr["skipped"])
+        achieved = k_bytes / (k_ms / 1e3) / 1e9
+        step_gbs = step_bytes / (ms_max / 1e3) / 1e9
+        return {
+            "workload": name, "description": wl["desc"], "psi": bn.psi, "nd": nd, "stage": wl["stage"],
+            "mode": {0: "speculative", 1: "two_pass", 2: "stash"}[mode], "owned_params": bn.owned,
+            "assembled_params": bn.assembled, "steps": steps, "skipped_steps": tr["skipped"],
+            "injected_steps": tr["injected"], "ms_per_step": ms_max / steps,
+            "params_per_s": world * bn.owned * steps / (ms_max / 1e3),
+            "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
+            "update_kernel_ms": k_ms,
+            "roofline": {"bound": "hbm", "kernel": update_kernel_name(nd, mode), "alg_bytes_per_launch": k_bytes,
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak},
+            "step": {"alg_bytes": step_bytes, "gbs": step_gbs, "frac": step_gbs / peak,
+                     "bytes": "applied steps: owned x (2 Nd + 26) + 4 x assembled; skipped steps: "
+                              "owned x 2 Nd"},
+            "gpu_launches": tr["launches"], "clocks": tr["clocks"],
+        }
+    finally:
+        bn.close()
+        del bn
+        torch.cuda.empty_cache()
+
+
+CONFIG_SWEEP = [(1 << 30, 1), (1 << 30, 8), (1 << 30, 64), (2 << 30, 1), (2 << 30, 8), (2 << 30, 64)]
+
+
+def run_configs(args, world: int, local: int, peak: float) -> list:
+    """The other named workloads and the sweep's >= 1B points, each allocated,
+    measured and freed in turn after the headline."""
+    import torch
+    wls = _workloads()
+    out = [config_entry("7.5b-nd64-stage3-owner0", wls["7.5b-nd64-stage3-owner0"], args, world, local,
+                        peak, seed=21),
+           config_entry("24l-d2048-stage2-nd16-clip", wls["24l-d2048-stage2-nd16-clip"], args, world, local,
+                        peak, seed=22, inject_rate=0.01)]
+    for psi, nd in CONFIG_SWEEP:
+        torch.cuda.empty_cache()
+        free, _ = torch.cuda.mem_get_info()
+        wl = sweep_workload(psi, nd, 1, int(max_over_ranks(-float(free), world) * -1))
+        e = config_entry(f"sweep-psi{psi}-nd{nd}-stage1", wl, args, world, local, peak, seed=23 + nd)
+        e["view"] = "owner0" if wl["owner_count"] == 1 else "all owners"
+        out.append(e)
+    return out
 
 
 SWEEP_PSI = [1 << 20, 16 << 20, 256 << 20, 1 << 30, 2 << 30]
@@ -601,6 +756,171 @@ def run_layer_gather(args) -> int:
     return 0
 
 
+LINK_GBS = 770.0   # measured peer copy per direction over NVLink 5 on this part (900 nominal)
+
+
+class HostTimer:
+    """Wall clock of a region on the host (the CPU harness tests' timer)."""
+
+    def start(self):
+        self.t0 = time.perf_counter()
+
+    def stop(self) -> float:
+        return (time.perf_counter() - self.t0) * 1e3
+
+
+class DeviceTimer:
+    """CUDA events on the current stream around a region."""
+
+    def __init__(self):
+        import torch
+        self.torch = torch
+        self.a = torch.cuda.Event(enable_timing=True)
+        self.b = torch.cuda.Event(enable_timing=True)
+
+    def start(self):
+        self.a.record()
+
+    def stop(self) -> float:
+        self.b.record()
+        self.torch.cuda.synchronize()
+        return self.a.elapsed_time(self.b)
+
+
+def sharded_loop(step, steps: int, warmup: int, world: int, timer, sync=lambda: None,
+                 device: str = "cuda") -> float:
+    """Warm-up, then ``steps`` calls of ``step(k)`` timed by ``timer``,
+    bracketed by a barrier and ``sync`` on both sides; returns the slowest
+    rank's ms (every rank takes the same collective steps)."""
+    for k in range(warmup):
+        step(-1 - k)
+    sync()
+    _barrier(world)
+    sync()
+    timer.start()
+    for k in range(steps):
+        step(k)
+    ms = timer.stop()
+    _barrier(world)
+    return max_over_ranks(ms, world, device)
+
+
+def sharded_report(psi: int, world: int, L: int, steps: int, ms_max: float, k_ms_max: float | None,
+                   transport: str, peak: float, comm: dict) -> dict:
+    """What a step with one owner per process moves, against its bounds.
+
+    Per process and step, the reduce-scatter's input sends (Nd-1) gradient
+    slices of L elements and receives as many; the all-gather sends the own
+    fp16 shard to the Nd-1 others and receives theirs: 2 (Nd-1) L elements,
+    4 (Nd-1) L bytes, each way -- the 2 Psi of stages 1 and 2 on the ring,
+    plus padding.  The link bound is those bytes at LINK_GBS per direction.
+    comm: zero_state_bytes' report of the same Psi, Nd and stage."""
+    elems = 2 * (world - 1) * L
+    link_bytes = 2 * elems
+    step_ms = ms_max / steps
+    link_ms = link_bytes / (LINK_GBS * 1e9) * 1e3
+    out = {
+        "transport": transport, "owners": world, "shard_len": L,
+        "exchange": {"elements_each_way": elems, "bytes_each_way": link_bytes,
+                     "link_gbs": LINK_GBS, "link_bound_ms": link_ms,
+                     "link_frac": (link_ms / step_ms) if step_ms > 0 else None},
+        "accounting": {"comm_elems_pages": comm["comm_elems"], "comm_elems_ring": comm["comm_elems_ring"],
+                       "exchanged_elems_each_way": elems,
+                       "exchanged_over_ring": (elems / comm["comm_elems_ring"])
+                       if comm["comm_elems_ring"] else None},
+        "step_ms": step_ms,
+    }
+    if k_ms_max is not None:
+        # the owner's update: Nd contributions in, master/m/v read and written, 16-bit out
+        k_bytes = L * (2 * world + 26)
+        gbs = k_bytes / (k_ms_max / 1e3) / 1e9
+        out["update"] = {"kernel_ms": k_ms_max, "alg_bytes": k_bytes, "gbs": gbs, "frac_of_hbm": gbs / peak,
+                         "note": "peer transport: the contributions of other ranks and the parameter "
+                                 "stores cross NVLink inside this kernel" if transport == "peer" else
+                                 "contributions already local after the exchange"}
+    return out
+
+
+def run_sharded(args) -> int:
+    """--sharded {nccl,peer} (under torchrun, one process per GPU): the ZeRO-DP
+    step with one owner per GPU -- ZeroDPStep (NCCL all-to-all, vote,
+    all-gather) or ZeroDPPeerStep (the exchange inside the step's kernels over
+    peer memory, no multicast).  Psi is fixed while the owners grow with the
+    GPU count, so the scaling is strong."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from zero_dp_partitioned_shard_b200 import binding as B
+    from zero_dp_partitioned_shard_b200 import distributed as D
+    from zero_dp_partitioned_shard_b200 import synth
+    world, rank, local = _dist()
+    if world == 1 and not dist.is_initialized():
+        dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    wl = _workloads()[args.workload]
+    if wl["layout"] != B.ZERO_GRADS_FULL:
+        raise SystemExit("--sharded runs the workloads with full per-rank gradients")
+    psi = args.psi or _psi_of(wl)
+    hp = B.hparams(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=wl["wd"], loss_scale=wl["S"],
+                   max_grad_norm=wl["clip"], mode=wl["mode"])
+    cls = D.ZeroDPStep if args.sharded == "nccl" else D.ZeroDPPeerStep
+    st = cls(psi, hp, stage=wl["stage"], bucket=wl["bucket"], align=wl["align"])
+    try:
+        master = torch.empty(psi, dtype=torch.float32, device="cuda")
+        synth.fill_normal_(master, seed=999, std=0.02)
+        st.load_master(master)
+        del master
+        grad = st.grads if args.sharded == "peer" else torch.empty(st.psi_pad, dtype=torch.float16,
+                                                                     device="cuda")
+        synth.fill_normal_(grad[:psi], seed=1000 + rank, std=1e-3, scale=wl["S"])
+        grad[psi:].zero_()
+        k_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+        for a, b in k_events:
+            a.record()
+            b.record()
+
+        def one(k):
+            evs = k_events[k] if k >= 0 else (None, None)
+            st.args.timing_events[0] = evs[0].cuda_event if evs[0] is not None else None
+            st.args.timing_events[1] = evs[1].cuda_event if evs[1] is not None else None
+            if args.sharded == "nccl":
+                st.step(grad)
+            else:
+                st.step()
+
+        clocks = ClockSampler(local)
+        clocks.start()
+        launches0 = B.zero_launch_count()
+        ms_max = sharded_loop(one, args.steps, args.warmup, world, DeviceTimer(), torch.cuda.synchronize)
+        launches = B.zero_launch_count() - launches0
+        clk = clocks.stop()
+        k_ms_max = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in k_events), world)
+        peak, peak_kind = measured_hbm_peak()
+        rep = sharded_report(psi, world, st.L, args.steps, ms_max, k_ms_max, args.sharded, peak,
+                             B.zero_state_bytes(psi, world, wl["stage"], wl["align"]))
+        res = B.step_result_from_bytes(st.result.cpu().numpy().tobytes())
+        line = {
+            "metric": METRIC, "value": psi * args.steps / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "description": wl["desc"], "psi": psi, "nd": world,
+                       "stage": wl["stage"], "sharded": args.sharded,
+                       "parallelism": f"ZeRO-DP over {world} process(es), one owner shard per GPU",
+                       "peak_source": f"{peak_kind} hbm_gbs (copy)"},
+            "sharded": rep, "gpu_launches": launches, "clocks": clk,
+            "last_step": {"overflow": res.overflow, "t": res.t},
+        }
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        st.close()
+        dist.destroy_process_group()
+    return 0
+
+
 def _psi_of(wl):
     return sum(wl["sizes"]()) if wl.get("sizes") else wl["psi"]
 
@@ -621,11 +941,16 @@ def main():
                     help="dynamic loss scaling (the scale in the device optimizer state)")
     ap.add_argument("--layer-gather", action="store_true",
                     help="measure the stage-3 per-layer gather schedule (forward + backward)")
+    ap.add_argument("--sharded", choices=["nccl", "peer"], default=None,
+                    help="one owner per GPU under torchrun: NCCL exchange, or the exchange inside the "
+                         "kernels over peer memory (not the default: the default runs replicas)")
     ap.add_argument("--retain", action="store_true",
                     help="stage-2 retention: reduce-scatter into kept 16-bit shards, then the step on them")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other named workloads and the >= 1B sweep points ('configs')")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--cpu-sample", type=int, default=1 << 22)
     ap.add_argument("--ref-sample", type=int, default=1 << 21)
@@ -642,6 +967,8 @@ def main():
         return run_sweep(args)
     if args.layer_gather:
         return run_layer_gather(args)
+    if args.sharded and args.impl == "ours":
+        return run_sharded(args)
     wls = _workloads()
     if args.workload not in wls:
         ap.error(f"unknown workload {args.workload}; choose from {sorted(wls)}")
@@ -659,33 +986,11 @@ def main():
     alg, moved = bytes_per_param(wl["nd"], wl["mode"])
 
     # --- device-resident timing ---
-    for _ in range(args.warmup):
-        bench.step()
-    n_ev = 4 if args.retain else 2
-    k_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(n_ev)) for _ in range(args.steps)]
-    for evs in k_events:    # create the CUDA events before handing their handles over
-        for ev in evs:
-            ev.record()
-    torch.cuda.synchronize()
-    _barrier(world)
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    launches0 = B.zero_launch_count()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record()
-    for k in range(args.steps):
-        bench.step(k_events[k])
-    t_end.record()
-    torch.cuda.synchronize()
-    launches = B.zero_launch_count() - launches0
-    clk = clocks.stop()
-    _barrier(world)
-    ms = t_start.elapsed_time(t_end)
+    tr = timed_steps(bench, args.steps, args.warmup, world, local, n_ev=4 if args.retain else 2)
+    ms, launches, clk = tr["ms_total"], tr["launches"], tr["clocks"]
     ms_max, value = aggregate(bench.owned, args.steps, ms, world)
-    k_ms = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in k_events)
-    r_ms = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in k_events) if args.retain else None
+    k_ms = statistics.mean(tr["kernel_ms"])
+    r_ms = statistics.mean(tr["reduce_ms"]) if args.retain else None
     k_ms_max = max_over_ranks(k_ms, world)
     res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
 
@@ -693,7 +998,7 @@ def main():
     e2e = None
     if not args.no_e2e:
         import psutil
-        need = bench.grad_bytes
+        need = bench.grad_bytes + bench.params.numel() * 2
         # every rank on this node pins its own copy; all ranks must agree on
         # running the leg, since it holds collectives (barrier, max over ranks)
         n_local = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
@@ -702,6 +1007,8 @@ def main():
         if fits:
             g_host = torch.empty(bench.grads.numel(), dtype=bench.grads.dtype, pin_memory=True)
             g_host.copy_(bench.grads)
+            # the step's product: the updated 16-bit parameters (the all-gathered buffer)
+            p_host = torch.empty(bench.params.numel(), dtype=bench.params.dtype, pin_memory=True)
             r_host = torch.empty(B.RESULT_BYTES, dtype=torch.uint8, pin_memory=True)
             torch.cuda.synchronize()
             for it in range(1 + args.e2e_steps):
@@ -712,6 +1019,7 @@ def main():
                     e0.record()
                 bench.grads.copy_(g_host, non_blocking=True)
                 bench.step()
+                p_host.copy_(bench.params, non_blocking=True)
                 r_host.copy_(bench.result, non_blocking=True)
                 torch.cuda.current_stream().synchronize()
                 B.step_result_from_bytes(r_host.numpy().tobytes())  # the caller reads the result
@@ -719,12 +1027,16 @@ def main():
             torch.cuda.synchronize()
             e_ms, e_value = aggregate(bench.owned, args.e2e_steps, e0.elapsed_time(e1), world)
             e2e = {"value": e_value, "unit": UNIT,
-                   "h2d_bytes_per_step": bench.grad_bytes, "d2h_bytes_per_step": B.RESULT_BYTES,
-                   "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps}
-            del g_host
+                   "h2d_bytes_per_step": bench.grad_bytes,
+                   "d2h_bytes_per_step": p_host.numel() * p_host.element_size() + B.RESULT_BYTES,
+                   "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
+                   "copies": "rank gradients host->device, updated 16-bit parameters and the "
+                             "result struct device->host, every step"}
+            del g_host, p_host
         else:
             e2e = {"value": None, "unit": UNIT,
-                   "skipped": "host memory below 2.5x the gradient bytes of every rank on the node"}
+                   "skipped": "host memory below 2.5x the gradient and parameter bytes of every rank "
+                              "on the node"}
 
     peak, peak_kind = measured_hbm_peak()
     k_bytes = bench.owned * update_launch_bytes(k_nd, wl["mode"], n_dests)
@@ -750,7 +1062,8 @@ def main():
                    "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
-                     "kernel": "zs_update_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "kernel": update_kernel_name(k_nd, wl["mode"], bool(n_dests)),
+                     "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
                      "alg_bytes_per_launch": k_bytes},
         "e2e": e2e,
@@ -765,11 +1078,16 @@ def main():
         line["retention"]["reduce_frac"] = line["retention"]["reduce_gbs"] / peak
         line["config"]["step_gbs_alg"] = (bench.owned * (2 * wl["nd"] + 2 + update_launch_bytes(1, wl["mode"]))
                                           / (ms_max / args.steps / 1e3) / 1e9)
+    bench.close()
+    del bench
+    torch.cuda.empty_cache()
+    if not (args.no_configs or args.psi or args.peer or args.retain or args.dynamic_scale
+            or args.storage != "fp16"):
+        line["configs"] = run_configs(args, world, local, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, args.cpu_sample,
                                             oracle.host_threads(), STORAGES[args.storage])
-    bench.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -66,3 +66,24 @@ def test_the_committed_profiles_carry_the_keys_the_lookup_reads():
     for name, kv in keys.items():
         assert set(kv) == {"traffic_bytes_per_param", "traffic_nd", "traffic_mode", "kernels_cu_sha256_prefix"}, name
         assert 0 < float(kv["traffic_bytes_per_param"]) < 200 and len(kv["kernels_cu_sha256_prefix"]) == 16
+
+
+def test_step_bytes_of_a_run_with_skipped_steps():
+    # applied steps: (2 Nd + 26) per owned parameter + 4 per assembled one
+    assert bench.step_alg_bytes(1000, 0, 8, 3, 0) == 3 * 1000 * 42
+    assert bench.step_alg_bytes(100, 6300, 64, 1, 0) == 100 * 154 + 4 * 6300
+    # a skipped step only read the contributions
+    assert bench.step_alg_bytes(1000, 0, 16, 20, 1) == 19 * 1000 * 58 + 1000 * 32
+    assert bench.step_alg_bytes(1000, 0, 16, 1, 1) == 1000 * 32
+
+
+def test_sharded_report_volumes():
+    comm = {"comm_elems": 2 * 1000, "comm_elems_ring": 2 * 1000 * 3 / 4}
+    rep = bench.sharded_report(1000, 4, 256, 10, 20.0, 0.5, "nccl", 6500.0, comm)
+    assert rep["exchange"]["elements_each_way"] == 2 * 3 * 256
+    assert rep["exchange"]["bytes_each_way"] == 4 * 3 * 256
+    assert rep["exchange"]["link_bound_ms"] == pytest.approx(4 * 3 * 256 / 770e9 * 1e3)
+    assert rep["accounting"]["exchanged_over_ring"] == pytest.approx(4 * 256 / 1000)
+    assert rep["step_ms"] == 2.0
+    assert rep["update"]["alg_bytes"] == 256 * (2 * 4 + 26)
+    assert rep["update"]["gbs"] == pytest.approx(256 * 34 / 0.5e-3 / 1e9)
