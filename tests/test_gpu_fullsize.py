@@ -336,22 +336,26 @@ def test_sweep_points_full_parity(psi, nd, stage):
     assert g.opt.t == o.opt.t == 1 and g.results[-1].t == 1
 
 
-@pytest.mark.parametrize("psi,nd,stage", [
-    (256 << 20, 1, 1),      # Nd <= 2: the low-byte streams
-    (256 << 20, 2, 2),      # ... in 8 buckets
-    (1 << 30, 64, 3),       # one owner of 64 at 1B (the one-owner view)
+@pytest.mark.parametrize("psi,nd,stage,mode", [
+    (256 << 20, 1, 1, 0),      # Nd <= 2: the low-byte streams
+    (256 << 20, 2, 2, 0),      # ... in 8 buckets
+    (1 << 30, 64, 3, 0),       # one owner of 64 at 1B (the one-owner view)
+    (64 << 20, 16, 1, 0),      # the pipelined update at its largest Nd
+    (64 << 20, 16, 2, 1),      # ... re-reducing in place after a clipped statistics pass
+    (48 << 20, 4, 3, 0),       # ... at Nd = 4, per-owner layout
+    ((32 << 20) - 8, 8, 1, 0), # just under the size from which Nd = 8 takes the pipeline
 ])
-def test_sweep_points_large_sampled(psi, nd, stage):
-    """The sweep's large points in the configuration the sweep times: every
-    owned element is updated on the GPU, sampled elements (random plus every
-    shard, bucket and vector boundary) are recomputed by the oracle from the
-    device bytes over two steps."""
+def test_sweep_points_large_sampled(psi, nd, stage, mode):
+    """The sweep's large points in the configuration the sweep times, and the
+    kernel choices around them: every owned element is updated on the GPU,
+    sampled elements (random plus every shard, bucket and vector boundary) are
+    recomputed by the oracle from the device bytes over two steps."""
     free, _ = torch.cuda.mem_get_info()
-    wl = bench.sweep_workload(psi, nd, stage, free)
+    wl = bench.sweep_workload(psi, nd, stage, free, mode)
     assert (wl["owner_count"] == 1) == (nd == 64)
     bn = bench.Bench(wl, None, seed=11 + nd)
     try:
-        res = _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=nd + stage)
+        res = _check_sampled_steps(bn, steps=2, n_random=1 << 19, seed=nd + stage, clip_from_gpu=mode != 0)
         assert [r.overflow for r in res] == [0, 0] and res[-1].t == 2
     finally:
         bn.close()

@@ -20,8 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libzero_shard.so")
 
-SOURCES = ["kernels.cu", "api.cpp", "plan.cpp", "static_scratch.cu", "peer.cpp"]
-HEADERS = [os.path.join(CSRC, "zs_internal.h"), os.path.join(INCLUDE, "zero_shard.h")]
+SOURCES = ["kernels.cu", "gather.cu", "api.cpp", "plan.cpp", "static_scratch.cu", "peer.cpp"]
+HEADERS = [os.path.join(CSRC, "zs_internal.h"), os.path.join(CSRC, "zs_launch.h"), os.path.join(INCLUDE, "zero_shard.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-fmad=false", "-Xcompiler", "-fPIC",

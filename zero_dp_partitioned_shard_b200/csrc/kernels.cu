@@ -45,6 +45,7 @@
 #include <utility>
 
 #include "zs_internal.h"
+#include "zs_launch.h"
 
 namespace zs {
 
@@ -1057,52 +1058,7 @@ zs_reduce_kernel(const uint16_t* grads, uint16_t* out, int nd, const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// K4: gather-assembly of fp16 parameter shards into the full buffer
-// ---------------------------------------------------------------------------
-
-// STREAM: evict-first loads and stores.  Measured: they suit the compact per-layer
-// gathers, whose two small buffers are rewritten every other layer (0.90 of
-// the copy peak against 0.86-0.88 with plain stores); plain write-back stores
-// suit the assembly of a full parameter buffer (0.94 against 0.92).
-template <bool STREAM>
-__global__ void __launch_bounds__(kThreads)
-zs_gather_kernel(uint16_t* dst, const __grid_constant__ GatherList g)
-{
-    // the pieces' units -- 8-element vectors for aligned pieces, single
-    // elements otherwise -- as one grid-stride index space (see walk_segments)
-    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-    int64_t total = 0;
-    for (int k = 0; k < g.count; ++k)
-        total += g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n;
-    int k = 0;
-    int64_t base = 0;
-    for (int64_t u = tid; u < total; u += nthr) {
-        while (u >= base + (g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n)) {
-            base += g.e[k].vec ? g.e[k].n >> 3 : g.e[k].n;
-            ++k;
-        }
-        const GatherEntry& ge = g.e[k];
-        const int64_t i = u - base;
-        if (ge.vec) {
-            uint4* to = reinterpret_cast<uint4*>(dst + ge.dst_off) + i;
-            if (STREAM)
-                __stcs(to, ld_stream(ge.src + (i << 3)));
-            else
-                *to = *reinterpret_cast<const uint4*>(ge.src + (i << 3));
-        } else
-            dst[ge.dst_off + i] = ge.src[i];
-    }
-    for (int j = 0; j < g.count; ++j) { // tails of the vector pieces
-        const GatherEntry& ge = g.e[j];
-        const int64_t e = ((ge.n >> 3) << 3) + tid;
-        if (ge.vec && e < ge.n)
-            dst[ge.dst_off + e] = ge.src[e];
-    }
-}
-
-// ---------------------------------------------------------------------------
-// launch geometry
+// launch geometry (the helpers shared with gather.cu are in zs_launch.h)
 // ---------------------------------------------------------------------------
 
 struct DevInfo {
@@ -1111,9 +1067,9 @@ struct DevInfo {
 
 static std::mutex g_mu;
 static std::unordered_map<int, DevInfo> g_dev;
-static std::map<std::pair<const void*, int>, int> g_occ; // (kernel, device) -> blocks per SM
+static std::map<std::pair<const void*, int>, int> g_occ; // (kernel, device or shape key) -> blocks per SM
 
-static cudaError_t device_sms(int* sms)
+cudaError_t device_sms(int* sms)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1132,39 +1088,29 @@ static cudaError_t device_sms(int* sms)
     return cudaSuccess;
 }
 
-// Persistent grid: SM count x resident blocks, but no more blocks than work.
-template <typename K>
-static cudaError_t grid_for(K kernel, int64_t work_threads, int cap, int* blocks)
+cudaError_t blocks_per_sm(const void* kernel, int* occ)
 {
-    int sms = 0;
-    cudaError_t e = device_sms(&sms);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess)
-        return e;
-    const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
-    int occ = 0;
+    const std::pair<const void*, int> key(kernel, dev);
     {
         std::lock_guard<std::mutex> lk(g_mu);
         auto it = g_occ.find(key);
-        if (it != g_occ.end())
-            occ = it->second;
+        if (it != g_occ.end()) {
+            *occ = it->second;
+            return cudaSuccess;
+        }
     }
-    if (occ == 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0);
-        if (e != cudaSuccess)
-            return e;
-        if (occ < 1)
-            occ = 1;
-        std::lock_guard<std::mutex> lk(g_mu);
-        g_occ[key] = occ;
-    }
-    int64_t want = (work_threads + kThreads - 1) / kThreads;
-    int64_t full = (int64_t)sms * occ;
-    if (cap > 0 && full > cap)
-        full = cap;
-    *blocks = (int)(want < 1 ? 1 : (want < full ? want : full));
+    int o = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kernel, kThreads, 0);
+    if (e != cudaSuccess)
+        return e;
+    o = o < 1 ? 1 : o;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_occ[key] = o;
+    *occ = o;
     return cudaSuccess;
 }
 
@@ -1180,51 +1126,6 @@ static int64_t seg_work(const SegList& s, bool vec)
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-
-// Every kernel launch of the library goes through here.  overlapped: with
-// programmatic stream serialization, so the kernel may begin while its
-// predecessor in the stream drains (it orders itself with
-// griddepcontrol.wait); used for the kernels after the first of a step.
-// While a prepare call is running (zs::preparing()) the kernel is only
-// loaded -- the caller has already resolved its geometry -- and nothing is
-// enqueued or counted.
-template <typename... Params, typename... Args>
-static cudaError_t launch_k(bool overlapped, void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
-                            cudaStream_t s, Args... args)
-{
-    if (preparing()) {
-        cudaFuncAttributes fa;
-        return cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(kernel));
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = overlapped ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
-    if (e == cudaSuccess)
-        count_launches(1);
-    return e;
-}
-
-template <typename... Params, typename... Args>
-static cudaError_t launch_overlapped(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
-                                     cudaStream_t s, Args... args)
-{
-    return launch_k(true, kernel, grid, block, smem, s, args...);
-}
-
-template <typename... Params, typename... Args>
-static cudaError_t launch_plain(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
-                                cudaStream_t s, Args... args)
-{
-    return launch_k(false, kernel, grid, block, smem, s, args...);
-}
 
 cudaError_t launch_opt_init(zero_opt_state* st, float scale, float growth, float backoff, int32_t interval,
                             cudaStream_t s)
@@ -1402,14 +1303,27 @@ static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const P
 
 // The bulk-copy pipeline takes the stash source and up to 16 contributions
 // (see pipe_shape for the measurements); the register path, whose groups of
-// 8 rank loads need no copy per rank, takes larger Nd.
-static bool use_pipeline(int src, int nd) { return src == kSrcStash || nd <= kPipeMaxNd; }
+// 8 rank loads need no copy per rank, takes larger Nd.  A launch of fewer
+// than 32M elements leaves each CTA under ~70 tiles, and the ring's fill and
+// drain then cost several percent: from Nd = 4 up, where the register path
+// is close at full speed, such launches take the register path (16M elements
+// at Nd = 8: 0.95 against 0.85 of the copy bandwidth).  With Nd <= 3 the
+// pipeline wins at every size (16M elements at Nd = 1: 0.89 against 0.77).
+constexpr int64_t kPipeMinElems = int64_t(1) << 25;
+
+static bool use_pipeline(int src, int nd, int64_t elems)
+{
+    if (src == kSrcStash)
+        return true;
+    return nd <= 3 || (nd <= kPipeMaxNd && elems >= kPipeMinElems);
+}
 
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
                           cudaStream_t s)
 {
     PipeShape ps;
-    if (vec && use_pipeline(src, a.nd) && (!peers || src == kSrcStash) && pipe_shape(src, a.nd, &ps)) {
+    if (vec && use_pipeline(src, a.nd, seg_work(segs, true) * 8) && (!peers || src == kSrcStash) &&
+        pipe_shape(src, a.nd, &ps)) {
         switch (src) {
         case kSrcGradsSpeculative: return launch_pipe<kSrcGradsSpeculative>(a, segs, ps, nullptr, s);
         case kSrcGradsInPlace: return launch_pipe<kSrcGradsInPlace>(a, segs, ps, nullptr, s);
@@ -1554,19 +1468,6 @@ cudaError_t launch_cast(bool vec, bool bf16, const float* master, uint16_t* para
     if (bf16)
         return vec ? launch_cast_t<true, true>(master, params, segs, s) : launch_cast_t<false, true>(master, params, segs, s);
     return vec ? launch_cast_t<true, false>(master, params, segs, s) : launch_cast_t<false, false>(master, params, segs, s);
-}
-
-cudaError_t launch_gather(uint16_t* dst, const GatherList& g, bool streaming_stores, cudaStream_t s)
-{
-    int64_t w = 0;
-    for (int i = 0; i < g.count; ++i)
-        w += g.e[i].vec ? (g.e[i].n + 7) >> 3 : g.e[i].n;
-    auto kernel = streaming_stores ? zs_gather_kernel<true> : zs_gather_kernel<false>;
-    int blocks = 0;
-    cudaError_t e = grid_for(kernel, w, 0, &blocks);
-    if (e != cudaSuccess)
-        return e;
-    return launch_plain(kernel, blocks, kThreads, 0, s, dst, g);
 }
 
 } // namespace zs

@@ -141,6 +141,7 @@ struct GatherList {
     int32_t count;
     int32_t pad;
     GatherEntry e[kMaxSegs];
+    int64_t first[kMaxSegs + 1]; // first unit of each piece, then the total (filled by launch_gather)
 };
 
 // ---- launchers (kernels.cu); each returns the launch's cudaError_t ----------
