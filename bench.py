@@ -15,8 +15,11 @@ measurement through the C-ABI call with the step's gradients copied from
 pinned host memory every step and the step's product (the updated 16-bit
 parameters) and its result struct copied back; ``roofline``
 reports the update kernel's algorithmic bytes per launch over its CUDA-event
-duration against the measured HBM copy bandwidth; ``cpu_baseline`` times the
-CPU oracle on a bounded sample on this host.
+duration against the measured HBM copy bandwidth; ``sustained`` repeats the
+step back to back for a few seconds and reports the update kernel over the
+last third, at the SM clock the power cap settles on; ``configs`` measures the
+other named workloads and the sweep's >= 1B points in the same run;
+``cpu_baseline`` times the CPU oracle on a bounded sample on this host.
 
 ``--peer`` runs the same step through peer tables with the Nd ranks' buffers
 in this GPU's memory: each rank's gradient read through the table, every new
@@ -99,11 +102,12 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     return alg, moved
 
 
-def update_kernel_name(nd: int, mode: int, peer: bool = False) -> str:
+def update_kernel_name(nd: int, mode: int, peer: bool = False, elems: int = 1 << 30) -> str:
     """The library's update kernel for this source: the bulk-copy pipeline for
-    the stash and up to 16 local contributions, the register path otherwise
-    (larger Nd, or contributions read through peer tables)."""
-    if mode == 2 or (nd <= 16 and not peer):
+    the stash and up to 16 local contributions (from Nd = 4 only for launches
+    of at least 32M elements), the register path otherwise (larger Nd, small
+    launches, or contributions read through peer tables)."""
+    if mode == 2 or (not peer and (nd <= 3 or (nd <= 16 and elems >= 1 << 25))):
         return "zs_update_pipe_kernel"
     return "zs_update_kernel"
 
@@ -554,7 +558,8 @@ def config_entry(name: str, wl: dict, args, world: int, local: int, peak: float,
             "params_per_s": world * bn.owned * steps / (ms_max / 1e3),
             "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
             "update_kernel_ms": k_ms,
-            "roofline": {"bound": "hbm", "kernel": update_kernel_name(nd, mode), "alg_bytes_per_launch": k_bytes,
+            "roofline": {"bound": "hbm", "kernel": update_kernel_name(nd, mode, False, bn.owned),
+                         "alg_bytes_per_launch": k_bytes,
                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak},
             "step": {"alg_bytes": step_bytes, "gbs": step_gbs, "frac": step_gbs / peak,
                      "bytes": "applied steps: owned x (2 Nd + 26) + 4 x assembled; skipped steps: "
@@ -946,6 +951,9 @@ def main():
                          "kernels over peer memory (not the default: the default runs replicas)")
     ap.add_argument("--retain", action="store_true",
                     help="stage-2 retention: reduce-scatter into kept 16-bit shards, then the step on them")
+    ap.add_argument("--sustained-seconds", type=float, default=3.0,
+                    help="after the timed steps, run the step back to back this long and report the update "
+                         "kernel at the clock the power cap settles on (0: skip)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -993,6 +1001,23 @@ def main():
     r_ms = statistics.mean(tr["reduce_ms"]) if args.retain else None
     k_ms_max = max_over_ranks(k_ms, world)
     res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
+
+    # --- sustained: the same step back to back for a few seconds, so that the
+    # power cap sets the SM clock as it does inside a training job ---
+    sustained = None
+    if args.sustained_seconds > 0:
+        n_sus = int(max_over_ranks(float(max(10, math.ceil(args.sustained_seconds * 1e3 / (ms / args.steps)))),
+                                   world))
+        ts = timed_steps(bench, n_sus, 0, world, local)
+        k_all = ts["kernel_ms"]
+        tail = k_all[len(k_all) * 2 // 3:]          # the last third: the settled clock
+        k_sus = max_over_ranks(statistics.mean(tail), world)
+        sus_bytes = bench.owned * update_launch_bytes(k_nd, wl["mode"], len(bench.dests))
+        sustained = {"seconds": max_over_ranks(ts["ms_total"], world) / 1e3, "steps": n_sus,
+                     "update_kernel_ms_last_third": k_sus,
+                     "update_kernel_ms_all": max_over_ranks(statistics.mean(k_all), world),
+                     "frac_last_third": sus_bytes / (k_sus / 1e3) / 1e9 / measured_hbm_peak()[0],
+                     "clocks": ts["clocks"]}
 
     # --- end to end through the C ABI, host buffers ---
     e2e = None
@@ -1062,11 +1087,12 @@ def main():
                    "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
-                     "kernel": update_kernel_name(k_nd, wl["mode"], bool(n_dests)),
+                     "kernel": update_kernel_name(k_nd, wl["mode"], bool(n_dests), bench.owned),
                      "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
                      "alg_bytes_per_launch": k_bytes},
         "e2e": e2e,
+        "sustained": sustained,
         "gpu_launches": launches,
         "clocks": clk,
         "last_step": {"overflow": res.overflow, "t": res.t},
