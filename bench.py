@@ -102,12 +102,28 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
     return alg, moved
 
 
+def pipeline_min_elems(nd: int, sms: int = 148) -> int:
+    """Smallest launch (elements) with which the library's pipelined update
+    gives every CTA 64 tiles, for 4 <= Nd <= 64: tiles of 256 x EPT elements,
+    SMs x CTAs per SM CTAs (the shapes of the library's pipe_shape)."""
+    if nd <= 16:
+        ept, ctas = 4, (3 if nd <= 12 else 2)
+    else:
+        e = 12 + 2 * nd
+        ept = 2 if 2 * (1024 + 2 * 256 * 2 * e + 1024) <= 228 * 1024 else 1
+        smem = 1024 + 2 * 256 * ept * e
+        ctas = 3
+        while ctas > 1 and ctas * (smem + 1024) > 228 * 1024:
+            ctas -= 1
+    return 64 * 256 * ept * sms * ctas
+
+
 def update_kernel_name(nd: int, mode: int, peer: bool = False, elems: int = 1 << 30) -> str:
     """The library's update kernel for this source: the bulk-copy pipeline for
-    the stash and up to 16 local contributions (from Nd = 4 only for launches
-    of at least 32M elements), the register path otherwise (larger Nd, small
-    launches, or contributions read through peer tables)."""
-    if mode == 2 or (not peer and (nd <= 3 or (nd <= 16 and elems >= 1 << 25))):
+    the stash and up to 64 local contributions (from Nd = 4 only for launches
+    that give every CTA at least 64 tiles), the register path otherwise
+    (larger Nd, small launches, or contributions read through peer tables)."""
+    if mode == 2 or (not peer and (nd <= 3 or (nd <= 64 and elems >= pipeline_min_elems(nd)))):
         return "zs_update_pipe_kernel"
     return "zs_update_kernel"
 

@@ -4,8 +4,9 @@
 // root and three divisions per parameter against 2*Nd + 26 bytes), so it uses
 // no tensor cores.  The update runs as a bulk-copy pipeline (warp-specialised:
 // one producer warp streams tiles into a shared-memory ring with
-// cp.async.bulk, eight consumer warps compute from it) for up to 16
-// contributions and for the stash, and on the register path below for more.
+// cp.async.bulk -- for more than 16 contributions as 2-D tensor-map boxes of
+// all rank rows -- and eight consumer warps compute from it) for up to 64
+// contributions and for the stash, and on the register path below otherwise.
 // Design points of the register path, which the statistics, reduce, commit
 // and cast kernels share:
 //   * one thread owns 8 consecutive parameters per iteration: every access is
@@ -35,6 +36,7 @@
 // intrinsic (no contraction into FMA), division and square root are the
 // IEEE-rounded __fdiv_rn / __fsqrt_rn, and the fp16 cast is round-to-nearest-
 // even with subnormals kept.
+#include <cuda.h> // CUtensorMap and the tensor-map encoder's types (the encoder is looked up at run time)
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -548,6 +550,26 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
+// global -> shared copy of one box of a 2-D tensor map (the box's top-left
+// element at column x, row y) completing as transaction bytes on `bar`.  The
+// whole box always lands in shared memory; elements past the map's extent
+// arrive as zeros.  x * 2 bytes must be a multiple of 16 (the host checks it
+// before the launch).  No multicast.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// The tensor map of a pipelined launch that moves the rank rows of a tile
+// with 2-D copies (TM), or nothing.
+struct NoMap {};
+template <bool TM>
+using TmapParam = typename std::conditional<TM, CUtensorMap, NoMap>::type;
+constexpr int kBoxCols = 256; // columns (elements) of one 2-D box; a tile of T elements takes T / 256 boxes
+
 template <int N>
 __device__ __forceinline__ void lds_f(const float* p, float f[N])
 {
@@ -616,20 +638,30 @@ __device__ __forceinline__ void stg_h(uint16_t* p, const float f[N])
     }
 }
 
-// tile g of the launch -> segment and offset, through the per-CTA tile table
-__device__ __forceinline__ int tile_segment(const int64_t* first_tile, int count, int64_t g)
+// Segment of tile g, through the per-CTA tile table.  A thread's tiles only
+// move forward (g += gridDim.x), so it keeps the segment of its previous tile
+// and advances from there: over a whole launch at most `count` steps, instead
+// of a scan of the table per tile (which, with one segment per owner of a
+// 64-owner call and 256-element tiles, cost as much as the arithmetic).
+__device__ __forceinline__ int next_tile_segment(const int64_t* first_tile, int count, int64_t g, int si)
 {
-    int s = 0;
-    while (s + 1 < count && g >= first_tile[s + 1])
-        ++s;
-    return s;
+    while (si + 1 < count && g >= first_tile[si + 1])
+        ++si;
+    return si;
 }
 
-template <int SRC, int EPT, bool BF, bool PEER>
+// TM: the Nd rank rows of a tile arrive as T / 256 two-dimensional boxes of
+// [256 columns x Nd rows] from a tensor map over the contributions (one copy
+// per box instead of one per rank); in shared memory box b holds rank r's
+// columns at (b * Nd + r) * 256.  Without TM each rank row is one 1-D copy
+// and rank r's row starts at r * T.
+template <int SRC, int EPT, bool BF, bool PEER, bool TM>
 __global__ void __launch_bounds__(kPipeThreads, 2)
 zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages,
-                      const __grid_constant__ PeerParam<PEER> pt)
+                      const __grid_constant__ PeerParam<PEER> pt, const __grid_constant__ TmapParam<TM> tmap)
 {
+    static_assert(!TM || (SRC != kSrcStash && !PEER && (kPipeConsumers * EPT) % kBoxCols == 0),
+                  "2-D boxes carry local rank rows of whole 256-column boxes");
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
     constexpr int T = kPipeConsumers * EPT; // elements per tile
     wait_for_predecessor();
@@ -677,8 +709,9 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
         // ---- producer warp: lane 0 claims a free stage and announces its
         // bytes; the tile's copies (3 state arrays + the source rows) are then
         // issued by all 32 lanes at once ----
-        const int n_copies = 3 + (SRC == kSrcStash ? 1 : a.nd);
+        const int n_copies = 3 + (SRC == kSrcStash ? 1 : (TM ? 1 : a.nd));
         int it = 0;
+        int si = 0; // segment of the current tile
         for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
             const int st = it % stages;
             bool ok = true;
@@ -688,14 +721,14 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 failed = true;
                 break;
             }
-            const int si = tile_segment(first_tile, segs.count, g);
+            si = next_tile_segment(first_tile, segs.count, g, si);
             const Seg& sg = segs.seg[si];
             const int64_t e0 = (g - first_tile[si]) * T;
             const int64_t nv = (sg.n >> 3) * 8;
             const uint32_t n = (uint32_t)(nv - e0 < T ? nv - e0 : T);
             unsigned char* buf = ring + (size_t)st * stage_bytes;
-            if (lane == 0)
-                mbar_arrive_expect_tx(&full[st], n * (12u + (uint32_t)src_bytes));
+            if (lane == 0) // 2-D boxes always deliver whole boxes, also past the tile's last element
+                mbar_arrive_expect_tx(&full[st], TM ? n * 12u + (uint32_t)(T * src_bytes) : n * (12u + (uint32_t)src_bytes));
             __syncwarp();
             const int64_t so = sg.s_off + e0;
             for (int j = lane; j < n_copies; j += 32) {
@@ -704,6 +737,15 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                     bulk_load(buf + j * (T * 4), src + so, n * 4, &full[st]);
                 } else if (SRC == kSrcStash) {
                     bulk_load(buf + T * 12, a.stash + so, n * 4, &full[st]);
+                } else if constexpr (TM) {
+                    // the tile's contributions start at column f % stride of
+                    // row f / stride (rank 0 of the segment's owner)
+                    const int64_t f = sg.g_off + e0;
+                    const int32_t x = (int32_t)(f % sg.g_rstride), y = (int32_t)(f / sg.g_rstride);
+#pragma unroll
+                    for (int b = 0; b < T / kBoxCols; ++b)
+                        tma_load_2d(buf + T * 12 + (size_t)b * kBoxCols * src_bytes, &tmap, x + b * kBoxCols, y,
+                                    &full[st]);
                 } else {
                     const int r = j - 3;
                     bulk_load(buf + T * 12 + r * (T * 2), ranks_at<PEER>(a.grads, pt, sg, e0).at(r), n * 2,
@@ -728,6 +770,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
         const int c = threadIdx.x; // 0 .. kPipeConsumers-1
         bool bad = false;
         int it = 0;
+        int si = 0; // segment of the current tile
         for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
             const int st = it % stages;
             const bool ok = mbar_wait(&full[st], (it / stages) & 1, a.wait_budget);
@@ -735,7 +778,7 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 failed = true;
                 break;
             }
-            const int si = tile_segment(first_tile, segs.count, g);
+            si = next_tile_segment(first_tile, segs.count, g, si);
             const Seg& sg = segs.seg[si];
             const int64_t e0 = (g - first_tile[si]) * T;
             const int64_t nv = (sg.n >> 3) * 8;
@@ -750,11 +793,15 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 if (SRC == kSrcStash) {
                     lds_f<EPT>(reinterpret_cast<const float*>(buf + T * 12) + i0, gr);
                 } else {
-                    const uint16_t* gs = reinterpret_cast<const uint16_t*>(buf + T * 12) + i0;
+                    // rank r's EPT elements: TM boxes hold 256 columns per
+                    // rank row; 1-D copies hold T
+                    const int rstep = TM ? kBoxCols : T;
+                    const uint16_t* gs = reinterpret_cast<const uint16_t*>(buf + T * 12) +
+                                         (TM ? (i0 / kBoxCols) * kBoxCols * a.nd + i0 % kBoxCols : i0);
                     lds_h<EPT, BF>(gs, gr);
                     for (int r = 1; r < a.nd; ++r) {
                         float f[EPT];
-                        lds_h<EPT, BF>(gs + r * T, f);
+                        lds_h<EPT, BF>(gs + r * rstep, f);
 #pragma unroll
                         for (int q = 0; q < EPT; ++q)
                             gr[q] = __fadd_rn(gr[q], f[q]);
@@ -1191,27 +1238,41 @@ static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegLi
 //     1.02 at Nd = 16 against 0.94-0.97 for the register path;
 //   * the 4-byte stash: EPT 8, 2 stages, 2 CTAs -- 0.96 against 0.89 for a
 //     3-stage ring and 0.92 for the register path.
+//   * contributions, 17 <= Nd <= 64: the Nd rank rows of a tile as 2-D
+//     tensor-map boxes of [256 columns x Nd rows] (one copy per box instead
+//     of one per rank, which at Nd = 32-64 had made the copy issue, not HBM,
+//     the limit: 0.60-0.64), 2 stages: 2 boxes per tile while two CTAs fit
+//     (Nd = 24: 3 CTAs, 1.01-1.04; Nd = 32: 2 CTAs, 0.99-1.01; Nd = 48:
+//     2 CTAs, 1.05), else 1 box per tile and 3 CTAs (Nd = 64: 1.00-1.02),
+//     against 0.91-0.99 for the register path.
 // A shallow ring with more CTAs per SM beat every deeper one: the same bytes
-// in flight per SM, spread over more independent producers.  Beyond Nd = 16
-// a tile needs Nd + 3 small copies and the copy issue, not HBM, limits the
-// pipeline (0.6 at Nd = 32 and 64); the register path takes those.
+// in flight per SM, spread over more independent producers.  Beyond Nd = 64
+// the register path takes over.
 struct PipeShape {
     int ept = 0, stages = 0, ctas_per_sm = 0, smem = 0;
+    bool tm = false; // rank rows by 2-D tensor-map boxes
 };
 
-constexpr int kPipeMaxNd = 16;
+constexpr int kPipeMaxNd = 16;    // 1-D copies of the rank rows up to here
+constexpr int kPipeMaxNdTm = 64;  // 2-D tensor-map boxes of all Nd rank rows up to here
 
 static bool pipe_shape(int src, int nd, PipeShape* ps)
 {
     const bool stash = src == kSrcStash;
-    if (!stash && nd > kPipeMaxNd)
+    if (!stash && nd > kPipeMaxNdTm)
         return false;
     const int e = 12 + (stash ? 4 : 2 * nd); // bytes per element of one stage
     PipeShape p;
     if (stash) {
         p.ept = 8, p.stages = 2, p.ctas_per_sm = 2;
-    } else {
+    } else if (nd <= kPipeMaxNd) {
         p.ept = 4, p.stages = 2, p.ctas_per_sm = 3;
+    } else {
+        // 2-D boxes of all Nd rank rows: two 256-column boxes per tile while a
+        // 2-stage ring of them still fits two CTAs per SM (Nd <= 50), else one
+        const int two_boxes = kPipeHeaderBytes + 2 * kPipeConsumers * 2 * e;
+        p.ept = 2 * (two_boxes + 1024) <= 228 * 1024 ? 2 : 1;
+        p.stages = 2, p.ctas_per_sm = 3, p.tm = true;
     }
     // CTAs per SM that the shared memory allows (228 KB per SM, 1 KB of it
     // reserved per CTA); the launch also checks the occupancy it gets
@@ -1229,11 +1290,82 @@ static bool pipe_shape(int src, int nd, PipeShape* ps)
 
 static std::map<std::pair<const void*, int>, int> g_smem_set; // (kernel, device) -> bytes allowed
 
-template <int SRC, int EPT, bool BF, bool PEER>
+// cuTensorMapEncodeTiled, looked up once from the driver through the runtime
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled()
+{
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// The tensor map of the rank rows a launch reads: a 2-D array of 16-bit
+// values whose row stride is the segments' rank stride, rows = ranks (of all
+// owners in the per-owner layout), boxes of [256 columns x Nd rows].  Its
+// extent is exactly the columns and rows the segments address, so a box's
+// overhang past a segment's end reads no memory (it arrives as zeros).
+// Returns false (and the launch takes the register path) unless every box
+// coordinate the kernel will use is a multiple of 8 columns (16 bytes) and
+// the map encodes.
+static bool rank_rows_map(const UpdateArgs& a, const SegList& segs, CUtensorMap* map)
+{
+    const EncodeTiledFn encode = encode_tiled();
+    if (!encode || segs.count < 1 || a.nd < 1 || a.nd > 256 || (reinterpret_cast<uintptr_t>(a.grads) & 15))
+        return false;
+    const int64_t stride = segs.seg[0].g_rstride;
+    if (stride <= 0 || stride % 8)
+        return false;
+    int64_t cols = 0, rows = 0;
+    for (int i = 0; i < segs.count; ++i) {
+        const Seg& sg = segs.seg[i];
+        if (sg.g_rstride != stride || sg.g_off < 0)
+            return false;
+        const int64_t x0 = sg.g_off % stride, y0 = sg.g_off / stride;
+        // tiles start at x0 + (multiples of 256): all on 16-byte columns
+        if (x0 % 8 || x0 + sg.n > stride)
+            return false;
+        cols = cols > x0 + sg.n ? cols : x0 + sg.n;
+        rows = rows > y0 + a.nd ? rows : y0 + a.nd;
+    }
+    if (cols < 1 || cols > INT32_MAX - 2 * kBoxCols || rows > INT32_MAX)
+        return false;
+    const cuuint64_t dim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t stride_bytes[1] = {(cuuint64_t)stride * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)a.nd};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(a.grads), dim, stride_bytes, box,
+                  elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool TM>
+static bool tmap_param(const UpdateArgs& a, const SegList& segs, TmapParam<TM>* out)
+{
+    if constexpr (TM)
+        return rank_rows_map(a, segs, out);
+    else
+        return true;
+}
+
+template <int SRC, int EPT, bool BF, bool PEER, bool TM>
 static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                  const PeerTable* peers, cudaStream_t s)
 {
-    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER>;
+    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER, TM>;
+    TmapParam<TM> tmap;
+    if (!tmap_param<TM>(a, segs, &tmap))
+        return cudaErrorNotSupported; // the caller falls back to the register path
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || (e = device_sms(&sms)) != cudaSuccess)
@@ -1274,16 +1406,21 @@ static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const
     grid = tiles < grid ? tiles : grid;
     grid = grid < 1 ? 1 : grid;
     return launch_overlapped(kernel, (unsigned)grid, kPipeThreads, ps.smem, s, a, segs, ps.stages,
-                             peer_param<PEER>(peers));
+                             peer_param<PEER>(peers), tmap);
 }
 
 template <int SRC, bool BF, bool PEER>
 static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                  const PeerTable* peers, cudaStream_t s)
 {
-    // pipe_shape chooses 8 (the stash) or 4 (contributions) elements per thread
-    return ps.ept == 8 ? launch_pipe_t<SRC, 8, BF, PEER>(a, segs, ps, peers, s)
-                       : launch_pipe_t<SRC, 4, BF, PEER>(a, segs, ps, peers, s);
+    // pipe_shape chooses 8 (the stash) or 4 (contributions, 1-D rows) elements
+    // per thread, or 1 or 2 (contributions by 2-D boxes)
+    if constexpr (SRC != kSrcStash && !PEER)
+        if (ps.tm)
+            return ps.ept == 2 ? launch_pipe_t<SRC, 2, BF, PEER, true>(a, segs, ps, peers, s)
+                               : launch_pipe_t<SRC, 1, BF, PEER, true>(a, segs, ps, peers, s);
+    return ps.ept == 8 ? launch_pipe_t<SRC, 8, BF, PEER, false>(a, segs, ps, peers, s)
+                       : launch_pipe_t<SRC, 4, BF, PEER, false>(a, segs, ps, peers, s);
 }
 
 // With peer tables the pipeline runs only from the stash (its rank loads stay
@@ -1301,34 +1438,40 @@ static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const P
                   : launch_pipe_f<SRC, false, false>(a, segs, ps, nullptr, s);
 }
 
-// The bulk-copy pipeline takes the stash source and up to 16 contributions
-// (see pipe_shape for the measurements); the register path, whose groups of
-// 8 rank loads need no copy per rank, takes larger Nd.  A launch of fewer
-// than 32M elements leaves each CTA under ~70 tiles, and the ring's fill and
-// drain then cost several percent: from Nd = 4 up, where the register path
-// is close at full speed, such launches take the register path (16M elements
-// at Nd = 8: 0.95 against 0.85 of the copy bandwidth).  With Nd <= 3 the
-// pipeline wins at every size (16M elements at Nd = 1: 0.89 against 0.77).
-constexpr int64_t kPipeMinElems = int64_t(1) << 25;
+// The bulk-copy pipeline takes the stash source and up to 64 contributions
+// (see pipe_shape for the measurements); the register path takes larger Nd,
+// and any launch whose layout a tensor map cannot describe with 16-byte
+// aligned columns.  A launch that leaves each CTA fewer than 64 tiles pays
+// several percent for the ring's fill and drain: from Nd = 4 up, where the
+// register path is close at full speed, such launches take the register path
+// (16M elements at Nd = 8, 37 tiles per CTA: 0.95 against 0.85 of the copy
+// bandwidth).  With Nd <= 3 the pipeline wins at every size (16M elements at
+// Nd = 1: 0.89 against 0.77).
+constexpr int64_t kPipeMinTilesPerCta = 64;
 
-static bool use_pipeline(int src, int nd, int64_t elems)
+static bool use_pipeline(int src, int nd, int64_t elems, const PipeShape& ps, int sms)
 {
-    if (src == kSrcStash)
+    if (src == kSrcStash || nd <= 3)
         return true;
-    return nd <= 3 || (nd <= kPipeMaxNd && elems >= kPipeMinElems);
+    const int64_t tiles = elems / ((int64_t)kPipeConsumers * ps.ept);
+    return nd <= kPipeMaxNdTm && tiles >= kPipeMinTilesPerCta * (int64_t)sms * ps.ctas_per_sm;
 }
 
 cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList& segs, const PeerTable* peers,
                           cudaStream_t s)
 {
     PipeShape ps;
-    if (vec && use_pipeline(src, a.nd, seg_work(segs, true) * 8) && (!peers || src == kSrcStash) &&
-        pipe_shape(src, a.nd, &ps)) {
+    int sms = 0;
+    if (vec && (!peers || src == kSrcStash) && pipe_shape(src, a.nd, &ps) && device_sms(&sms) == cudaSuccess &&
+        use_pipeline(src, a.nd, seg_work(segs, true) * 8, ps, sms)) {
+        cudaError_t e;
         switch (src) {
-        case kSrcGradsSpeculative: return launch_pipe<kSrcGradsSpeculative>(a, segs, ps, nullptr, s);
-        case kSrcGradsInPlace: return launch_pipe<kSrcGradsInPlace>(a, segs, ps, nullptr, s);
-        default: return launch_pipe<kSrcStash>(a, segs, ps, peers, s);
+        case kSrcGradsSpeculative: e = launch_pipe<kSrcGradsSpeculative>(a, segs, ps, nullptr, s); break;
+        case kSrcGradsInPlace: e = launch_pipe<kSrcGradsInPlace>(a, segs, ps, nullptr, s); break;
+        default: e = launch_pipe<kSrcStash>(a, segs, ps, peers, s); break;
         }
+        if (e != cudaErrorNotSupported) // not a tensor-map launch the layout allows: register path
+            return e;
     }
     switch (src) {
     case kSrcGradsSpeculative: return launch_update_regs<kSrcGradsSpeculative>(vec, a, segs, peers, s);
