@@ -120,10 +120,11 @@ def pipeline_min_elems(nd: int, sms: int = 148) -> int:
 
 def update_kernel_name(nd: int, mode: int, peer: bool = False, elems: int = 1 << 30) -> str:
     """The library's update kernel for this source: the bulk-copy pipeline for
-    the stash and up to 64 local contributions (from Nd = 4 only for launches
-    that give every CTA at least 64 tiles), the register path otherwise
-    (larger Nd, small launches, or contributions read through peer tables)."""
-    if mode == 2 or (not peer and (nd <= 3 or (nd <= 64 and elems >= pipeline_min_elems(nd)))):
+    the stash, and for up to 64 contributions (up to 16 through peer tables;
+    from Nd = 4 only for launches that give every CTA at least 64 tiles); the
+    register path otherwise (larger Nd, small launches)."""
+    max_nd = 16 if peer else 64
+    if mode == 2 or nd <= 3 or (nd <= max_nd and elems >= pipeline_min_elems(nd)):
         return "zs_update_pipe_kernel"
     return "zs_update_kernel"
 
@@ -451,6 +452,21 @@ def _draw_grads(storage: int):
     return synth.grads_bf16 if storage == 1 else synth.grads_f16
 
 
+def host_cpu() -> dict:
+    """The host's logical CPU count and model name (from /proc/cpuinfo; None
+    where it is not readable)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cpus": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(wl: dict, budget_s: float, sample_psi: int, threads: int, storage: int = 0) -> dict:
     """The CPU oracle, as it stands, on a bounded sample of the workload."""
     import oracle
@@ -475,7 +491,7 @@ def cpu_baseline(wl: dict, budget_s: float, sample_psi: int, threads: int, stora
     return {"value": sample_psi * steps / el, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{steps} oracle steps over {sample_psi:,} params x Nd={nd} "
                       f"(same hyper-parameters), {el:.1f} s, OpenMP threads={threads}",
-            "gbs_alg": sample_psi * steps * alg / el / 1e9}
+            "gbs_alg": sample_psi * steps * alg / el / 1e9, **host_cpu()}
 
 
 def run_reference(args, wl_name: str, wl: dict):
@@ -513,7 +529,7 @@ def run_reference(args, wl_name: str, wl: dict):
         "config": {"workload": wl_name, "description": wl["desc"], "psi": _psi_of(wl),
                    "nd": nd, "storage": args.storage, "sample_params_per_step": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": f"{args.steps} steps over {sample:,} params x Nd={nd}"},
+                         "sample": f"{args.steps} steps over {sample:,} params x Nd={nd}", **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -1016,6 +1032,7 @@ def main():
     k_ms = statistics.mean(tr["kernel_ms"])
     r_ms = statistics.mean(tr["reduce_ms"]) if args.retain else None
     k_ms_max = max_over_ranks(k_ms, world)
+    k_ms_median = max_over_ranks(statistics.median(tr["kernel_ms"]), world)
     res = B.step_result_from_bytes(bench.result.cpu().numpy().tobytes())
 
     # --- sustained: the same step back to back for a few seconds, so that the
@@ -1106,6 +1123,7 @@ def main():
                      "kernel": update_kernel_name(k_nd, wl["mode"], bool(n_dests), bench.owned),
                      "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
+                     "kernel_ms_median": k_ms_median,
                      "alg_bytes_per_launch": k_bytes},
         "e2e": e2e,
         "sustained": sustained,

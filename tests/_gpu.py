@@ -208,3 +208,15 @@ def to_oracle_hp(hp: B.HParams, storage: int = B.ZERO_STORAGE_FP16) -> oracle.HP
                      weight_decay=hp.weight_decay, loss_scale=hp.loss_scale,
                      max_grad_norm=hp.max_grad_norm, average_over_nd=bool(hp.average_over_nd),
                      storage=storage)
+
+
+def kernels_launched(fn):
+    """Runs fn() and returns (its result, the names of the CUDA kernels it
+    launched), recorded by the torch profiler's CUDA activity trace, which
+    sees the kernels of every library in the process."""
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        out = fn()
+        torch.cuda.synchronize()
+    names = {e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA}
+    return out, names

@@ -87,3 +87,9 @@ def test_sharded_report_volumes():
     assert rep["step_ms"] == 2.0
     assert rep["update"]["alg_bytes"] == 256 * (2 * 4 + 26)
     assert rep["update"]["gbs"] == pytest.approx(256 * 34 / 0.5e-3 / 1e9)
+
+
+def test_host_cpu_reports_count_and_model():
+    h = bench.host_cpu()
+    assert h["host_cpus"] == os.cpu_count()
+    assert h["cpu_model"] is None or isinstance(h["cpu_model"], str)

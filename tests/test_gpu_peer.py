@@ -14,8 +14,8 @@ import numpy as np
 import pytest
 import torch
 
-from _gpu import (CANARY, INF16, NAN16, PARAM_SENTINEL, STATE_SENTINEL, dev, host, make_problem,
-                  run_gpu, run_oracle, to_oracle_hp)
+from _gpu import (CANARY, INF16, NAN16, PARAM_SENTINEL, STATE_SENTINEL, dev, host, kernels_launched,
+                  make_problem, run_gpu, run_oracle, to_oracle_hp)
 from _util import assert_bf16_close, assert_f16_close, assert_f32_close
 from zero_dp_partitioned_shard_b200 import binding as B
 
@@ -228,6 +228,41 @@ def test_peer_tables_equal_the_strided_call(mode):
         assert np.array_equal(P, g.params)
     for a, b in ((master, g.master), (m, g.exp_avg), (v, g.exp_avg_sq)):
         assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+@pytest.fixture(scope="module")
+def pipeline_sized_problem():
+    psi = 33_554_437
+    pb = make_problem(psi, 8, align=256, steps=3, seed=66, S=1024.0, random_state=True)
+    pb.grads[1][5, 7 * (psi // 8) + 1234] = INF16[B.ZERO_STORAGE_FP16]
+    return pb
+
+
+@pytest.mark.parametrize("mode", MODES, ids=lambda m: MODE_NAMES[m])
+def test_peer_pipeline_launch(mode, pipeline_sized_problem):
+    """One call over all 8 owners, large enough for the bulk-copy pipeline
+    (at least 64 tiles of 1024 elements per CTA at 3 CTAs on each of 148
+    SMs: 29,097,984 elements), so the producer copies every rank row from its
+    own table entry and the consumers store into all 8 parameter buffers.
+    Ragged Psi, an inf in the second step: bit-identical to the strided call
+    on the same data, and within the oracle's bars."""
+    pb = pipeline_sized_problem
+    hp = B.hparams(loss_scale=1024.0, weight_decay=0.01, mode=mode,
+                   max_grad_norm=0.0 if mode == 0 else 0.05)
+    (params, master, m, v, C), names = kernels_launched(lambda: run_peer(pb, hp, per_rank=False))
+    if torch.cuda.get_device_properties(0).multi_processor_count <= 148:
+        assert any("zs_update_pipe_kernel" in n for n in names), sorted(names)
+        # the kernel the bench line names for this launch is the one that ran
+        import bench
+        assert any(bench.update_kernel_name(8, mode, True, pb.psi) in n for n in names), sorted(names)
+    assert [r.overflow for r in C[0]["results"]] == [0, 1, 0]
+    g = run_gpu(pb, hp, stage=2)
+    for P in params:
+        assert np.array_equal(P, g.params)
+    for a, b in ((master, g.master), (m, g.exp_avg), (v, g.exp_avg_sq)):
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    o = run_oracle(pb, to_oracle_hp(hp), clip_overrides=None if mode == 0 else [r.clip_coef for r in C[0]["results"]])
+    check(pb, hp, params, master, m, v, C, o, f"peer pipeline {MODE_NAMES[mode]}")
 
 
 @pytest.mark.parametrize("mode", MODES, ids=lambda m: MODE_NAMES[m])

@@ -1415,33 +1415,39 @@ static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const
 {
     // pipe_shape chooses 8 (the stash) or 4 (contributions, 1-D rows) elements
     // per thread, or 1 or 2 (contributions by 2-D boxes)
-    if constexpr (SRC != kSrcStash && !PEER)
-        if (ps.tm)
+    if (ps.tm) {
+        if constexpr (SRC != kSrcStash && !PEER)
             return ps.ept == 2 ? launch_pipe_t<SRC, 2, BF, PEER, true>(a, segs, ps, peers, s)
                                : launch_pipe_t<SRC, 1, BF, PEER, true>(a, segs, ps, peers, s);
+        // one tensor map cannot span the separate buffers of a peer table,
+        // and the 1-D kernel's tile does not fit a 2-D shape's ring
+        return cudaErrorNotSupported;
+    }
+    if (ps.ept != 8 && ps.ept != 4)
+        return cudaErrorNotSupported;
     return ps.ept == 8 ? launch_pipe_t<SRC, 8, BF, PEER, false>(a, segs, ps, peers, s)
                        : launch_pipe_t<SRC, 4, BF, PEER, false>(a, segs, ps, peers, s);
 }
 
-// With peer tables the pipeline runs only from the stash (its rank loads stay
-// on the register path); the stash pipeline then stores to every destination.
+// With peer tables the producer copies rank r's rows from table entry r (a
+// buffer of this GPU or another GPU's, by plain 1-D bulk copies: no
+// multicast), and the consumers store the new parameters into every
+// destination.
 template <int SRC>
 static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                const PeerTable* peers, cudaStream_t s)
 {
-    if constexpr (SRC == kSrcStash) {
-        if (peers)
-            return a.bf16 ? launch_pipe_f<SRC, true, true>(a, segs, ps, peers, s)
-                          : launch_pipe_f<SRC, false, true>(a, segs, ps, peers, s);
-    }
+    if (peers)
+        return a.bf16 ? launch_pipe_f<SRC, true, true>(a, segs, ps, peers, s)
+                      : launch_pipe_f<SRC, false, true>(a, segs, ps, peers, s);
     return a.bf16 ? launch_pipe_f<SRC, true, false>(a, segs, ps, nullptr, s)
                   : launch_pipe_f<SRC, false, false>(a, segs, ps, nullptr, s);
 }
 
 // The bulk-copy pipeline takes the stash source and up to 64 contributions
-// (see pipe_shape for the measurements); the register path takes larger Nd,
-// and any launch whose layout a tensor map cannot describe with 16-byte
-// aligned columns.  A launch that leaves each CTA fewer than 64 tiles pays
+// (see pipe_shape for the measurements), or up to 16 through peer tables
+// (1-D row copies only); the register path takes larger Nd, and any launch
+// whose layout a tensor map cannot describe with 16-byte aligned columns.  A launch that leaves each CTA fewer than 64 tiles pays
 // several percent for the ring's fill and drain: from Nd = 4 up, where the
 // register path is close at full speed, such launches take the register path
 // (16M elements at Nd = 8, 37 tiles per CTA: 0.95 against 0.85 of the copy
@@ -1449,10 +1455,12 @@ static cudaError_t launch_pipe(const UpdateArgs& a, const SegList& segs, const P
 // Nd = 1: 0.89 against 0.77).
 constexpr int64_t kPipeMinTilesPerCta = 64;
 
-static bool use_pipeline(int src, int nd, int64_t elems, const PipeShape& ps, int sms)
+static bool use_pipeline(int src, int nd, int64_t elems, const PipeShape& ps, int sms, bool peers)
 {
     if (src == kSrcStash || nd <= 3)
         return true;
+    if (peers && nd > kPipeMaxNd)
+        return false;
     const int64_t tiles = elems / ((int64_t)kPipeConsumers * ps.ept);
     return nd <= kPipeMaxNdTm && tiles >= kPipeMinTilesPerCta * (int64_t)sms * ps.ctas_per_sm;
 }
@@ -1462,15 +1470,15 @@ cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList&
 {
     PipeShape ps;
     int sms = 0;
-    if (vec && (!peers || src == kSrcStash) && pipe_shape(src, a.nd, &ps) && device_sms(&sms) == cudaSuccess &&
-        use_pipeline(src, a.nd, seg_work(segs, true) * 8, ps, sms)) {
+    if (vec && pipe_shape(src, a.nd, &ps) && device_sms(&sms) == cudaSuccess &&
+        use_pipeline(src, a.nd, seg_work(segs, true) * 8, ps, sms, peers != nullptr)) {
         cudaError_t e;
         switch (src) {
-        case kSrcGradsSpeculative: e = launch_pipe<kSrcGradsSpeculative>(a, segs, ps, nullptr, s); break;
-        case kSrcGradsInPlace: e = launch_pipe<kSrcGradsInPlace>(a, segs, ps, nullptr, s); break;
+        case kSrcGradsSpeculative: e = launch_pipe<kSrcGradsSpeculative>(a, segs, ps, peers, s); break;
+        case kSrcGradsInPlace: e = launch_pipe<kSrcGradsInPlace>(a, segs, ps, peers, s); break;
         default: e = launch_pipe<kSrcStash>(a, segs, ps, peers, s); break;
         }
-        if (e != cudaErrorNotSupported) // not a tensor-map launch the layout allows: register path
+        if (e != cudaErrorNotSupported) // a shape or tensor map this launch cannot take: register path
             return e;
     }
     switch (src) {
