@@ -105,7 +105,9 @@ def bytes_per_param(nd: int, mode: int) -> tuple[int, int]:
 def pipeline_min_elems(nd: int, sms: int = 148) -> int:
     """Smallest launch (elements) with which the library's pipelined update
     gives every CTA 64 tiles, for 4 <= Nd <= 64: tiles of 256 x EPT elements,
-    SMs x CTAs per SM CTAs (the shapes of the library's pipe_shape)."""
+    SMs x CTAs per SM CTAs (the shapes of the library's pipe_shape; the
+    2-byte result region of the bulk-store shapes, Nd 5-11, still leaves room
+    for 3 CTAs)."""
     if nd <= 16:
         ept, ctas = 4, (3 if nd <= 12 else 2)
     else:

@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import oracle
-from _gpu import (PARAM_SENTINEL, dev, host, make_problem, run_gpu, run_oracle, to_oracle_hp)
+from _gpu import (INF16, PARAM_SENTINEL, dev, host, kernels_launched, make_problem, run_gpu, run_oracle,
+                  to_oracle_hp)
 from _util import assert_f16_close, assert_f32_close
 from zero_dp_partitioned_shard_b200 import binding as B
 from zero_dp_partitioned_shard_b200 import synth
@@ -338,3 +339,33 @@ def test_dynamic_loss_scaling_sequence(mode, layout):
     assert [r.overflow for r in g.results] == [0, 0, 1, 0, 0, 1, 0, 0]
     assert [r.loss_scale for r in g.results] == [info["loss_scale"] for info in o.infos]
     assert [r.loss_scale for r in g.results] == [S0, 2 * S0, S0, S0, 2 * S0, S0, S0, 2 * S0]
+
+
+@pytest.fixture(scope="module")
+def bulk_store_problem():
+    psi = 32_000_017
+    pb = make_problem(psi, 6, align=256, steps=3, seed=71, S=1024.0, random_state=True)
+    pb.grads[1][2, 5 * (psi // 6) + 4321] = INF16[B.ZERO_STORAGE_FP16]
+    return pb
+
+
+@pytest.mark.parametrize("mode", [B.ZERO_MODE_SPECULATIVE, B.ZERO_MODE_TWO_PASS], ids=["speculative", "two_pass"])
+@pytest.mark.parametrize("layout", [B.ZERO_GRADS_FULL, B.ZERO_GRADS_PER_OWNER], ids=["full", "per_owner"])
+def test_bulk_store_pipeline_launch(mode, layout, bulk_store_problem):
+    """A pipelined update whose results leave through shared memory and the
+    producer's bulk stores (5 <= Nd <= 11 from the contributions): Nd = 6,
+    32,000,017 parameters in one call over all owners (70 tiles of 1024
+    elements per CTA at 3 CTAs on each of 148 SMs), six owner segments with
+    ragged ends, an overflow in the second of three steps; every element
+    against the oracle."""
+    pb = bulk_store_problem
+    hp = B.hparams(loss_scale=1024.0, weight_decay=0.01, mode=mode,
+                   max_grad_norm=0.0 if mode == B.ZERO_MODE_SPECULATIVE else 0.05)
+    stage = 3 if layout == B.ZERO_GRADS_PER_OWNER else 1
+    g, names = kernels_launched(lambda: run_gpu(pb, hp, layout=layout, stage=stage))
+    if torch.cuda.get_device_properties(0).multi_processor_count <= 148:
+        assert any("zs_update_pipe_kernel" in n for n in names), sorted(names)
+    assert [r.overflow for r in g.results] == [0, 1, 0]
+    o = run_oracle(pb, to_oracle_hp(hp),
+                   clip_overrides=None if mode == B.ZERO_MODE_SPECULATIVE else [r.clip_coef for r in g.results])
+    compare(g, o, f"bulk-store pipeline {MODE_NAMES[mode]} layout {layout}")

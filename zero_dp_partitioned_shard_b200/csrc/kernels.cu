@@ -541,13 +541,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     return true;
 }
 
-// global -> shared bulk copy of `bytes` (multiple of 16, both ends 16-byte
-// aligned) completing as transaction bytes on `bar`.  No multicast.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+// L2 policy of the 1-D pipeline's copies: evict first, like its streaming
+// stores.  Each byte is read once, so the lines it would keep in L2 are better
+// left to the dirty lines of the stores.  Measured on one B200 against the
+// default policy: GPT-2 1.5B-shaped Nd = 8 update 0.970-0.972 -> 0.974-0.975
+// of the copy bandwidth, and the 24-layer clip step (stash mode) 13.58 ->
+// 13.37-13.39 ms; with plain stores instead of evict-first ones the same
+// policy cost 3 % everywhere.  The tensor-map instantiations keep the default
+// policy: with evict-first copies Nd = 64 fell from 1.01-1.03 to 0.90-0.91.
+__device__ __forceinline__ uint64_t evict_first_policy()
 {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// global -> shared bulk copy of `bytes` (multiple of 16, both ends 16-byte
+// aligned) completing as transaction bytes on `bar`; with HINT under L2 policy
+// `pol`, else under the default policy.  No multicast.
+template <bool HINT>
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol)
+{
+    if constexpr (HINT)
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+                     " [%0], [%1], %2, [%3], %4;"
+                     ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+                     : "memory");
+    else
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                     : "memory");
 }
 
 // global -> shared copy of one box of a 2-D tensor map (the box's top-left
@@ -561,6 +584,45 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
                  " [%0], [%1, {%2, %3}], [%4];"
                  ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
                  : "memory");
+}
+
+// shared -> global bulk copy of `bytes` (multiple of 16, both ends 16-byte
+// aligned) under L2 policy `pol`, tracked by the issuing thread's bulk-async
+// groups.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes, uint64_t pol)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
+                 ::"l"(dst), "r"(smem_addr(src)), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void sts_f(float* p, const float f[N])
+{
+    if (N == 8) {
+        reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+        reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+    } else if (N == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+    } else if (N == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(f[0], f[1]);
+    } else {
+        p[0] = f[0];
+    }
+}
+
+template <int N, bool BF>
+__device__ __forceinline__ void sts_h(uint16_t* p, const float f[N])
+{
+    if (N == 8) {
+        *reinterpret_cast<uint4*>(p) = pack_h8<BF>(f);
+    } else if (N == 4) {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_h2<BF>(f[0], f[1]), pack_h2<BF>(f[2], f[3]));
+    } else if (N == 2) {
+        *reinterpret_cast<unsigned int*>(p) = pack_h2<BF>(f[0], f[1]);
+    } else {
+        p[0] = f2h<BF>(f[0]);
+    }
 }
 
 // The tensor map of a pipelined launch that moves the rank rows of a tile
@@ -655,13 +717,19 @@ __device__ __forceinline__ int next_tile_segment(const int64_t* first_tile, int 
 // per box instead of one per rank); in shared memory box b holds rank r's
 // columns at (b * Nd + r) * 256.  Without TM each rank row is one 1-D copy
 // and rank r's row starts at r * T.
-template <int SRC, int EPT, bool BF, bool PEER, bool TM>
+// BST: the consumers write a tile's results into the stage -- master/m/v over
+// their own input slots, the 16-bit parameters into a region of T * 2 bytes
+// after the source rows -- and the producer warp stores the tile with bulk
+// copies before it refills the stage.  Otherwise each consumer stores its own
+// results to global memory.
+template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST>
 __global__ void __launch_bounds__(kPipeThreads, 2)
 zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages,
                       const __grid_constant__ PeerParam<PEER> pt, const __grid_constant__ TmapParam<TM> tmap)
 {
     static_assert(!TM || (SRC != kSrcStash && !PEER && (kPipeConsumers * EPT) % kBoxCols == 0),
                   "2-D boxes carry local rank rows of whole 256-column boxes");
+    static_assert(!BST || (!TM && !PEER && SRC != kSrcStash), "bulk stores: 1-D contributions, no peer tables");
     constexpr bool kSpec = SRC == kSrcGradsSpeculative;
     constexpr int T = kPipeConsumers * EPT; // elements per tile
     wait_for_predecessor();
@@ -676,7 +744,8 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
     int64_t* first_tile = reinterpret_cast<int64_t*>(smem + 256); // [count + 1]
     unsigned char* ring = smem + kPipeHeaderBytes;
     const int src_bytes = SRC == kSrcStash ? 4 : 2 * a.nd;        // per element
-    const int stage_bytes = T * (12 + src_bytes);
+    const int params_off = T * (12 + src_bytes);                   // BST: the tile's 16-bit results
+    const int stage_bytes = T * (12 + src_bytes) + (BST ? T * 2 : 0);
 
     if (threadIdx.x == 0) {
         int64_t acc = 0;
@@ -710,6 +779,28 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
         // bytes; the tile's copies (3 state arrays + the source rows) are then
         // issued by all 32 lanes at once ----
         const int n_copies = 3 + (SRC == kSrcStash ? 1 : (TM ? 1 : a.nd));
+        constexpr bool kHint = !TM; // evict-first copies, except with tensor maps
+        const uint64_t pol = kHint ? evict_first_policy() : 0;
+        // BST: lane 0, which acquired the stage's empty barrier, stores the
+        // results of tile gw from the stage and waits until the copies have
+        // read shared memory, so that the stage can take new copies
+        int si_out = 0; // segment of the tile being stored
+        auto store_tile = [&](const unsigned char* sbuf, int64_t gw) {
+            if (lane == 0) {
+                si_out = next_tile_segment(first_tile, segs.count, gw, si_out);
+                const Seg& sw = segs.seg[si_out];
+                const int64_t w0 = (gw - first_tile[si_out]) * T;
+                const int64_t wv = (sw.n >> 3) * 8;
+                const uint32_t wn = (uint32_t)(wv - w0 < T ? wv - w0 : T);
+                bulk_store(p_out + sw.s_off + w0, sbuf, wn * 4, pol);
+                bulk_store(m_out + sw.s_off + w0, sbuf + T * 4, wn * 4, pol);
+                bulk_store(v_out + sw.s_off + w0, sbuf + T * 8, wn * 4, pol);
+                bulk_store(a.params + sw.p_off + w0, sbuf + params_off, wn * 2, pol);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            }
+            __syncwarp();
+        };
         int it = 0;
         int si = 0; // segment of the current tile
         for (int64_t g = blockIdx.x; g < n_tiles; g += gridDim.x, ++it) {
@@ -721,6 +812,9 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                 failed = true;
                 break;
             }
+            if constexpr (BST)
+                if (it >= stages) // the stage's previous tile
+                    store_tile(ring + (size_t)st * stage_bytes, g - (int64_t)stages * gridDim.x);
             si = next_tile_segment(first_tile, segs.count, g, si);
             const Seg& sg = segs.seg[si];
             const int64_t e0 = (g - first_tile[si]) * T;
@@ -734,9 +828,9 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
             for (int j = lane; j < n_copies; j += 32) {
                 if (j < 3) {
                     const float* src = j == 0 ? p_in : (j == 1 ? m_in : v_in);
-                    bulk_load(buf + j * (T * 4), src + so, n * 4, &full[st]);
+                    bulk_load<kHint>(buf + j * (T * 4), src + so, n * 4, &full[st], pol);
                 } else if (SRC == kSrcStash) {
-                    bulk_load(buf + T * 12, a.stash + so, n * 4, &full[st]);
+                    bulk_load<kHint>(buf + T * 12, a.stash + so, n * 4, &full[st], pol);
                 } else if constexpr (TM) {
                     // the tile's contributions start at column f % stride of
                     // row f / stride (rank 0 of the segment's owner)
@@ -748,10 +842,26 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
                                     &full[st]);
                 } else {
                     const int r = j - 3;
-                    bulk_load(buf + T * 12 + r * (T * 2), ranks_at<PEER>(a.grads, pt, sg, e0).at(r), n * 2,
-                              &full[st]);
+                    bulk_load<kHint>(buf + T * 12 + r * (T * 2), ranks_at<PEER>(a.grads, pt, sg, e0).at(r), n * 2,
+                                     &full[st], pol);
                 }
             }
+        }
+        if constexpr (BST) {
+            // the last tile of each stage, once its consumers are done
+            for (int j = it - stages < 0 ? 0 : it - stages; j < it && !failed; ++j) {
+                const int st = j % stages;
+                bool ok = true;
+                if (lane == 0)
+                    ok = mbar_wait(&empty[st], (j / stages) & 1, a.wait_budget);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    failed = true;
+                    break;
+                }
+                store_tile(ring + (size_t)st * stage_bytes, blockIdx.x + (int64_t)j * gridDim.x);
+            }
+            if (lane == 0) // the stores are complete before the CTA exits
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         }
         // every copy issued lands before the producer may leave the CTA
         if (lane == 0) {
@@ -818,14 +928,25 @@ zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, 
 #pragma unroll
                 for (int q = 0; q < EPT; ++q)
                     adam_update(kSpec ? gr[q] : __fmul_rn(gr[q], k.clip), p[q], m[q], v[q], k);
-                const int64_t so = sg.s_off + e0 + i0;
-                stg_f<EPT>(p_out + so, p);
-                stg_f<EPT>(m_out + so, m);
-                stg_f<EPT>(v_out + so, v);
-                stg_h<EPT, BF>(a.params + sg.p_off + e0 + i0, p);
-                if constexpr (PEER)
-                    for (int d = 0; d < pt.n_dests; ++d)
-                        stg_h<EPT, BF>(pt.dests[d] + sg.p_off + e0 + i0, p);
+                if constexpr (BST) {
+                    // this thread's own slots (it alone read them), made
+                    // visible to the producer's bulk copies
+                    unsigned char* wbuf = ring + (size_t)st * stage_bytes;
+                    sts_f<EPT>(reinterpret_cast<float*>(wbuf) + i0, p);
+                    sts_f<EPT>(reinterpret_cast<float*>(wbuf + T * 4) + i0, m);
+                    sts_f<EPT>(reinterpret_cast<float*>(wbuf + T * 8) + i0, v);
+                    sts_h<EPT, BF>(reinterpret_cast<uint16_t*>(wbuf + params_off) + i0, p);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                } else {
+                    const int64_t so = sg.s_off + e0 + i0;
+                    stg_f<EPT>(p_out + so, p);
+                    stg_f<EPT>(m_out + so, m);
+                    stg_f<EPT>(v_out + so, v);
+                    stg_h<EPT, BF>(a.params + sg.p_off + e0 + i0, p);
+                    if constexpr (PEER)
+                        for (int d = 0; d < pt.n_dests; ++d)
+                            stg_h<EPT, BF>(pt.dests[d] + sg.p_off + e0 + i0, p);
+                }
             }
             __syncwarp();
             if (lane == 0)
@@ -1248,25 +1369,40 @@ static cudaError_t launch_update_regs(bool vec, const UpdateArgs& a, const SegLi
 // A shallow ring with more CTAs per SM beat every deeper one: the same bytes
 // in flight per SM, spread over more independent producers.  Beyond Nd = 64
 // the register path takes over.
+// Stores (1-D contributions without peer tables): for 5 <= Nd <= 11 the
+// results leave through the stage and the producer's bulk copies (BST).  A/B
+// at 1B parameters, fractions of the copy bandwidth without -> with: Nd 5
+// 0.97 -> 0.98, 6 0.97 -> 1.00, 7 0.97 -> 1.01, 8 0.97-0.98 -> 1.01 (256M:
+// 0.94 -> 1.02, 2B: 0.97 -> 1.02), 9-11 0.96-0.97 -> 1.03-1.04.  Elsewhere
+// the consumers store directly: at Nd = 4 bulk stores read 0.93 against
+// 0.99, at Nd = 12 the results region leaves room for 2 CTAs only (0.93
+// against 0.98), at Nd = 16 0.99 against 1.05, at Nd = 1 0.87 against 0.98,
+// for the stash 0.91 against 0.98 and through peer tables 0.95 against 0.98:
+// the producer may refill a stage only once its stores have read it, which
+// costs more than it gains on streams with a larger share of writes.
 struct PipeShape {
     int ept = 0, stages = 0, ctas_per_sm = 0, smem = 0;
-    bool tm = false; // rank rows by 2-D tensor-map boxes
+    bool tm = false;  // rank rows by 2-D tensor-map boxes
+    bool bst = false; // results stored by the producer's bulk copies
 };
 
 constexpr int kPipeMaxNd = 16;    // 1-D copies of the rank rows up to here
 constexpr int kPipeMaxNdTm = 64;  // 2-D tensor-map boxes of all Nd rank rows up to here
+constexpr int kBulkStMinNd = 5, kBulkStMaxNd = 11; // bulk stores for these Nd (1-D, no peer tables)
 
-static bool pipe_shape(int src, int nd, PipeShape* ps)
+static bool pipe_shape(int src, int nd, bool peers, PipeShape* ps)
 {
     const bool stash = src == kSrcStash;
     if (!stash && nd > kPipeMaxNdTm)
         return false;
-    const int e = 12 + (stash ? 4 : 2 * nd); // bytes per element of one stage
+    int e = 12 + (stash ? 4 : 2 * nd); // bytes per element of one stage
     PipeShape p;
     if (stash) {
         p.ept = 8, p.stages = 2, p.ctas_per_sm = 2;
     } else if (nd <= kPipeMaxNd) {
         p.ept = 4, p.stages = 2, p.ctas_per_sm = 3;
+        p.bst = !peers && nd >= kBulkStMinNd && nd <= kBulkStMaxNd;
+        e += p.bst ? 2 : 0; // the 16-bit results region
     } else {
         // 2-D boxes of all Nd rank rows: two 256-column boxes per tile while a
         // 2-stage ring of them still fits two CTAs per SM (Nd <= 50), else one
@@ -1358,11 +1494,11 @@ static bool tmap_param(const UpdateArgs& a, const SegList& segs, TmapParam<TM>* 
         return true;
 }
 
-template <int SRC, int EPT, bool BF, bool PEER, bool TM>
+template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST = false>
 static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                  const PeerTable* peers, cudaStream_t s)
 {
-    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER, TM>;
+    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER, TM, BST>;
     TmapParam<TM> tmap;
     if (!tmap_param<TM>(a, segs, &tmap))
         return cudaErrorNotSupported; // the caller falls back to the register path
@@ -1425,6 +1561,12 @@ static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const
     }
     if (ps.ept != 8 && ps.ept != 4)
         return cudaErrorNotSupported;
+    if (ps.bst) {
+        if constexpr (SRC != kSrcStash && !PEER)
+            if (ps.ept == 4)
+                return launch_pipe_t<SRC, 4, BF, PEER, false, true>(a, segs, ps, peers, s);
+        return cudaErrorNotSupported;
+    }
     return ps.ept == 8 ? launch_pipe_t<SRC, 8, BF, PEER, false>(a, segs, ps, peers, s)
                        : launch_pipe_t<SRC, 4, BF, PEER, false>(a, segs, ps, peers, s);
 }
@@ -1470,7 +1612,7 @@ cudaError_t launch_update(int src, bool vec, const UpdateArgs& a, const SegList&
 {
     PipeShape ps;
     int sms = 0;
-    if (vec && pipe_shape(src, a.nd, &ps) && device_sms(&sms) == cudaSuccess &&
+    if (vec && pipe_shape(src, a.nd, peers != nullptr, &ps) && device_sms(&sms) == cudaSuccess &&
         use_pipeline(src, a.nd, seg_work(segs, true) * 8, ps, sms, peers != nullptr)) {
         cudaError_t e;
         switch (src) {
