@@ -1070,6 +1070,9 @@ def main():
             # the step's product: the updated 16-bit parameters (the all-gathered buffer)
             p_host = torch.empty(bench.params.numel(), dtype=bench.params.dtype, pin_memory=True)
             r_host = torch.empty(B.RESULT_BYTES, dtype=torch.uint8, pin_memory=True)
+            main = torch.cuda.current_stream()
+            side = torch.cuda.Stream()  # the parameter copy of step k beside the gradient copy of step k+1
+            p_done = None
             torch.cuda.synchronize()
             for it in range(1 + args.e2e_steps):
                 if it == 1:
@@ -1078,11 +1081,20 @@ def main():
                     e1 = torch.cuda.Event(enable_timing=True)
                     e0.record()
                 bench.grads.copy_(g_host, non_blocking=True)
+                if p_done is not None:
+                    main.wait_event(p_done)  # the step rewrites the parameters the last copy reads
                 bench.step()
-                p_host.copy_(bench.params, non_blocking=True)
                 r_host.copy_(bench.result, non_blocking=True)
-                torch.cuda.current_stream().synchronize()
+                stepped = torch.cuda.Event()
+                stepped.record(main)
+                with torch.cuda.stream(side):
+                    side.wait_event(stepped)
+                    p_host.copy_(bench.params, non_blocking=True)
+                    p_done = torch.cuda.Event()
+                    p_done.record(side)
+                main.synchronize()
                 B.step_result_from_bytes(r_host.numpy().tobytes())  # the caller reads the result
+            main.wait_event(p_done)  # the last step's parameters are on the host
             e1.record()
             torch.cuda.synchronize()
             e_ms, e_value = aggregate(bench.owned, args.e2e_steps, e0.elapsed_time(e1), world)
@@ -1091,7 +1103,8 @@ def main():
                    "d2h_bytes_per_step": p_host.numel() * p_host.element_size() + B.RESULT_BYTES,
                    "steps": args.e2e_steps, "ms_per_step": e_ms / args.e2e_steps,
                    "copies": "rank gradients host->device, updated 16-bit parameters and the "
-                             "result struct device->host, every step"}
+                             "result struct device->host, every step; the parameter copy of "
+                             "step k runs on a second stream beside the gradient copy of step k+1"}
             del g_host, p_host
         else:
             e2e = {"value": None, "unit": UNIT,
