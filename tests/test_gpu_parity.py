@@ -369,3 +369,41 @@ def test_bulk_store_pipeline_launch(mode, layout, bulk_store_problem):
     o = run_oracle(pb, to_oracle_hp(hp),
                    clip_overrides=None if mode == B.ZERO_MODE_SPECULATIVE else [r.clip_coef for r in g.results])
     compare(g, o, f"bulk-store pipeline {MODE_NAMES[mode]} layout {layout}")
+
+
+@pytest.mark.parametrize("nd", [5, 11])
+def test_bulk_store_pipeline_range_ends(nd):
+    """The ends of the bulk-store range: Nd = 5, and Nd = 11, whose results
+    region still leaves room for 3 CTAs per SM (2 ring stages of 1024
+    elements x 36 B).  29,600,003 parameters (just over 64 tiles per CTA),
+    two steps, every element against the oracle."""
+    pb = make_problem(29_600_003, nd, align=256, steps=2, seed=72 + nd, S=1024.0, random_state=True)
+    hp = B.hparams(loss_scale=1024.0, weight_decay=0.01, mode=B.ZERO_MODE_SPECULATIVE)
+    g, names = kernels_launched(lambda: run_gpu(pb, hp))
+    if torch.cuda.get_device_properties(0).multi_processor_count <= 148:
+        assert any("zs_update_pipe_kernel" in n for n in names), sorted(names)
+    compare(g, run_oracle(pb, to_oracle_hp(hp)), f"bulk-store pipeline Nd = {nd}")
+
+
+@pytest.mark.parametrize("psi,nd,mode", [
+    (30_000_000, 8, B.ZERO_MODE_SPECULATIVE),   # pipeline (>= 29.1M at 3 CTAs)
+    (16_000_000, 8, B.ZERO_MODE_SPECULATIVE),   # register path (under 64 tiles per CTA)
+    (1_000_000, 2, B.ZERO_MODE_SPECULATIVE),    # pipeline at any size for Nd <= 3
+    (2_000_000, 4, B.ZERO_MODE_STASH),          # the stash always takes the pipeline
+    (15_000_000, 17, B.ZERO_MODE_SPECULATIVE),  # tensor-map pipeline (>= 14.5M at Nd = 17)
+    (8_000_000, 17, B.ZERO_MODE_SPECULATIVE),   # register path
+])
+def test_bench_names_the_update_kernel_that_runs(psi, nd, mode):
+    """The bench line's roofline names its update kernel from the library's
+    shape rules; the kernel a launch of that size actually runs is the one
+    it names."""
+    import bench
+    pb = make_problem(psi, nd, align=256, steps=1, seed=73, S=1024.0)
+    hp = B.hparams(loss_scale=1024.0, mode=mode, max_grad_norm=0.0 if mode == B.ZERO_MODE_SPECULATIVE else 1.0)
+    _, names = kernels_launched(lambda: run_gpu(pb, hp))
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the shape rules are stated for 148 SMs")
+    want = bench.update_kernel_name(nd, mode, False, psi)
+    other = "zs_update_kernel" if want == "zs_update_pipe_kernel" else "zs_update_pipe_kernel"
+    assert any(want + "<" in n or want + "I" in n for n in names), sorted(names)
+    assert not any(other + "<" in n or other + "I" in n for n in names), sorted(names)
