@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import oracle
-from _gpu import INF16, NAN16, PARAM_SENTINEL, dev, host, make_problem, run_gpu, run_oracle, to_oracle_hp
+from _gpu import (INF16, NAN16, PARAM_SENTINEL, dev, host, kernels_launched, make_problem, run_gpu, run_oracle,
+                  to_oracle_hp)
 from _util import assert_bf16_close, assert_f32_close
 from zero_dp_partitioned_shard_b200 import binding as B
 from zero_dp_partitioned_shard_b200 import synth
@@ -55,8 +56,9 @@ def test_tiny_workload_bf16(mode, stage):
     assert g.opt.t == 3
 
 
-# (psi, nd, align, bucket): vectorised Nd <= 16 and the stash mode take the
-# bulk-copy pipeline; Nd = 64 the register path; align 1 the scalar path
+# (psi, nd, align, bucket): vectorised Nd <= 3 and the stash mode take the
+# bulk-copy pipeline at these sizes, the others the register path; align 1
+# the scalar path
 RAGGED = [(1, 1, 1, 0), (7, 3, 1, 0), (4097, 2, 8, 1000), (100_003, 1, 256, 0), (100_003, 7, 16, 4096),
           (200_001, 64, 256, 8192), (65_539, 2, 1, 0)]
 
@@ -166,3 +168,18 @@ def test_storage_formats_differ_only_in_rounding():
     ga, gb = run_gpu(a, hp), run_gpu(b, hp)
     assert not np.array_equal(ga.master, gb.master)
     assert_f32_close(gb.master, run_oracle(b, to_oracle_hp(hp, BF)).master, 2, "bf16")
+
+
+@pytest.mark.parametrize("psi,nd", [(30_000_007, 8), (15_000_011, 17)], ids=["bulk_stores_nd8", "tensor_map_nd17"])
+def test_pipeline_launches_bf16(psi, nd):
+    """Launches large enough for the bulk-copy pipeline with bfloat16
+    storage: Nd = 8 (results through the producer's bulk stores; 29,097,984
+    elements give 64 tiles per CTA) and Nd = 17 (rank rows as 2-D tensor-map
+    boxes; 14,548,992 elements).  Two steps, every element against the
+    oracle run with the same storage format."""
+    pb = make_problem(psi, nd, align=256, steps=2, seed=91 + nd, S=1.0, random_state=True, storage=BF)
+    hp = B.hparams(lr=1e-3, weight_decay=0.01, loss_scale=1.0, mode=B.ZERO_MODE_SPECULATIVE)
+    g, names = kernels_launched(lambda: run_gpu(pb, hp))
+    if torch.cuda.get_device_properties(0).multi_processor_count <= 148:
+        assert any("zs_update_pipe_kernel" in n for n in names), sorted(names)
+    compare(g, run_oracle(pb, to_oracle_hp(hp, BF)), f"bf16 pipeline Nd = {nd}")
