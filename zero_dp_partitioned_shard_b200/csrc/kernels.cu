@@ -722,8 +722,8 @@ __device__ __forceinline__ int next_tile_segment(const int64_t* first_tile, int 
 // after the source rows -- and the producer warp stores the tile with bulk
 // copies before it refills the stage.  Otherwise each consumer stores its own
 // results to global memory.
-template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST>
-__global__ void __launch_bounds__(kPipeThreads, 2)
+template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST, int MINB = 2>
+__global__ void __launch_bounds__(kPipeThreads, MINB)
 zs_update_pipe_kernel(const UpdateArgs a, const __grid_constant__ SegList segs, int stages,
                       const __grid_constant__ PeerParam<PEER> pt, const __grid_constant__ TmapParam<TM> tmap)
 {
@@ -1384,11 +1384,18 @@ struct PipeShape {
     int ept = 0, stages = 0, ctas_per_sm = 0, smem = 0;
     bool tm = false;  // rank rows by 2-D tensor-map boxes
     bool bst = false; // results stored by the producer's bulk copies
+    bool occ3 = false; // peer tables: the build bounded to 3 CTAs per SM
 };
 
 constexpr int kPipeMaxNd = 16;    // 1-D copies of the rank rows up to here
 constexpr int kPipeMaxNdTm = 64;  // 2-D tensor-map boxes of all Nd rank rows up to here
 constexpr int kBulkStMinNd = 5, kBulkStMaxNd = 11; // bulk stores for these Nd (1-D, no peer tables)
+// Peer tables: the kernel that stores into every destination needs 74
+// registers, which leave room for 2 CTAs per SM; a build bounded to 3 CTAs
+// (61 registers) is used up to this Nd.  One-GPU emulation, 512M parameters,
+// fraction of the copy bandwidth, 2-CTA -> 3-CTA build: Nd 1 0.86 -> 0.99,
+// Nd 2 0.87 -> 0.98, Nd 3 0.92 -> 0.96, Nd 4 0.97 -> 0.93, Nd 8 0.97 -> 0.92.
+constexpr int kPeerOcc3MaxNd = 3;
 
 static bool pipe_shape(int src, int nd, bool peers, PipeShape* ps)
 {
@@ -1402,6 +1409,7 @@ static bool pipe_shape(int src, int nd, bool peers, PipeShape* ps)
     } else if (nd <= kPipeMaxNd) {
         p.ept = 4, p.stages = 2, p.ctas_per_sm = 3;
         p.bst = !peers && nd >= kBulkStMinNd && nd <= kBulkStMaxNd;
+        p.occ3 = peers && nd <= kPeerOcc3MaxNd;
         e += p.bst ? 2 : 0; // the 16-bit results region
     } else {
         // 2-D boxes of all Nd rank rows: two 256-column boxes per tile while a
@@ -1494,11 +1502,11 @@ static bool tmap_param(const UpdateArgs& a, const SegList& segs, TmapParam<TM>* 
         return true;
 }
 
-template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST = false>
+template <int SRC, int EPT, bool BF, bool PEER, bool TM, bool BST = false, int MINB = 2>
 static cudaError_t launch_pipe_t(const UpdateArgs& a, const SegList& segs, const PipeShape& ps,
                                  const PeerTable* peers, cudaStream_t s)
 {
-    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER, TM, BST>;
+    auto kernel = zs_update_pipe_kernel<SRC, EPT, BF, PEER, TM, BST, MINB>;
     TmapParam<TM> tmap;
     if (!tmap_param<TM>(a, segs, &tmap))
         return cudaErrorNotSupported; // the caller falls back to the register path
@@ -1561,6 +1569,9 @@ static cudaError_t launch_pipe_f(const UpdateArgs& a, const SegList& segs, const
     }
     if (ps.ept != 8 && ps.ept != 4)
         return cudaErrorNotSupported;
+    if constexpr (PEER && SRC != kSrcStash)
+        if (ps.occ3 && ps.ept == 4)
+            return launch_pipe_t<SRC, 4, BF, PEER, false, false, 3>(a, segs, ps, peers, s);
     if (ps.bst) {
         if constexpr (SRC != kSrcStash && !PEER)
             if (ps.ept == 4)
