@@ -5,8 +5,10 @@
 // no tensor cores.  The update runs as a bulk-copy pipeline (warp-specialised:
 // one producer warp streams tiles into a shared-memory ring with
 // cp.async.bulk -- for more than 16 contributions as 2-D tensor-map boxes of
-// all rank rows -- and eight consumer warps compute from it) for up to 64
-// contributions and for the stash, and on the register path below otherwise.
+// all rank rows -- and eight consumer warps compute from it; for 5 to 11
+// contributions the results go back through the ring and leave by the
+// producer's bulk stores) for up to 64 contributions (16 through peer
+// tables) and for the stash, and on the register path below otherwise.
 // Design points of the register path, which the statistics, reduce, commit
 // and cast kernels share:
 //   * one thread owns 8 consecutive parameters per iteration: every access is
