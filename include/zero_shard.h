@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SHARD_ABI_VERSION 8
+#define ZERO_SHARD_ABI_VERSION 9
 
 /* Every entry point is exported with default visibility; the library hides
  * everything else. */
@@ -533,6 +533,14 @@ ZERO_API const char* zero_strerror(zero_status status);
 ZERO_API const char* zero_last_error(void);
 /* Number of kernels this library has launched in this process. */
 ZERO_API uint64_t zero_launch_count(void);
+/* Names of the kernels this library launched last in this process (up to the
+ * last 64 launches, from all threads), oldest first, as the compiler emits
+ * them (mangled C++ names, e.g. containing "zs_update_pipe_kernel"): writes
+ * up to `max` pointers into `names` (host array) and returns how many.  The
+ * strings belong to the CUDA runtime and stay valid while the library is
+ * loaded.  Returns -1 if max < 0, or if max > 0 and names is NULL.  For
+ * diagnostics and tests: which update kernel a call's shape rules chose. */
+ZERO_API int32_t zero_recent_kernels(const char** names, int32_t max);
 /* Budget, in SM clock cycles, of each bounded wait inside the pipelined
  * update kernel (default 2^31, about a second).  A wait that exceeds it makes
  * the step report status ZERO_ERR_TIMEOUT instead of hanging.  A negative

@@ -210,19 +210,13 @@ def to_oracle_hp(hp: B.HParams, storage: int = B.ZERO_STORAGE_FP16) -> oracle.HP
                      storage=storage)
 
 
-def kernels_launched(fn, attempts: int = 3):
-    """Runs fn() and returns (its result, the names of the CUDA kernels it
-    launched), recorded by the torch profiler's CUDA activity trace, which
-    sees the kernels of every library in the process.  fn must launch a step
-    (every step launches one update kernel): a trace holding no update kernel
-    at all has lost events, and fn is run again, at most `attempts` times."""
-    from torch.profiler import ProfilerActivity, profile
-    out, names = None, set()
-    for _ in range(attempts):
-        with profile(activities=[ProfilerActivity.CUDA], acc_events=True) as prof:
-            out = fn()
-            torch.cuda.synchronize()
-        names = {e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA}
-        if any("zs_update_kernel" in n or "zs_update_pipe_kernel" in n for n in names):
-            break
-    return out, names
+def kernels_launched(fn):
+    """Runs fn() and returns (its result, the names of the kernels of this
+    library that it launched), from the library's own launch record
+    (zero_recent_kernels: mangled C++ names, up to the last 64 launches)."""
+    before = B.zero_launch_count()
+    out = fn()
+    torch.cuda.synchronize()
+    n = B.zero_launch_count() - before
+    assert 0 < n <= 64, f"{n} launches: the record holds the last 64"
+    return out, set(B.zero_recent_kernels(n))

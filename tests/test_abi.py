@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
     lib = B.lib()
     for name in declared:
         assert getattr(lib, name) is not None
-    assert B.zero_abi_version() == 8
+    assert B.zero_abi_version() == 9
     # nothing else leaks out of the library (hidden visibility)
     assert all(n.startswith("zero_") for n in exported if not n.startswith("_"))
 
@@ -425,3 +425,14 @@ def test_plain_c_caller_links_and_calls_the_library(tmp_path):
                     "-L", pkg, "-lzero_shard", "-Wl,-rpath," + pkg], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
+
+
+def test_recent_kernels_record_arguments():
+    """zero_recent_kernels: argument checks, and nothing recorded before the
+    first launch of the process (the CPU suite launches no kernel)."""
+    lib = B.lib()
+    assert lib.zero_recent_kernels(None, -1) == -1
+    assert lib.zero_recent_kernels(None, 4) == -1
+    assert lib.zero_recent_kernels(None, 0) == 0
+    if B.zero_launch_count() == 0:
+        assert B.zero_recent_kernels() == []

@@ -154,6 +154,7 @@ SIGNATURES = {
     "zero_strerror": (C.c_char_p, [_S]),
     "zero_last_error": (C.c_char_p, []),
     "zero_launch_count": (C.c_uint64, []),
+    "zero_recent_kernels": (C.c_int32, [C.POINTER(C.c_char_p), C.c_int32]),
     "zero_set_wait_budget": (C.c_int64, [C.c_int64]),
 }
 
@@ -171,7 +172,7 @@ def lib() -> C.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        if L.zero_abi_version() != 8:
+        if L.zero_abi_version() != 9:
             raise ImportError("libzero_shard.so ABI version mismatch")
         _lib = L
     return _lib
@@ -352,6 +353,16 @@ def zero_last_error() -> str:
 
 def zero_launch_count() -> int:
     return lib().zero_launch_count()
+
+
+def zero_recent_kernels(max_names: int = 64) -> list:
+    """Names of the kernels the library launched last (oldest first, mangled
+    C++ names), up to the last 64 launches in the process."""
+    buf = (C.c_char_p * max_names)()
+    n = lib().zero_recent_kernels(buf, max_names)
+    if n < 0:
+        raise ValueError("zero_recent_kernels: bad arguments")
+    return [buf[i].decode() for i in range(n)]
 
 
 def zero_set_wait_budget(cycles: int) -> int:

@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <new>
 
 #include "zs_internal.h"
@@ -33,6 +34,19 @@ zero_status fail(zero_status s, const char* fmt, ...)
 void clear_error() { g_last_error[0] = '\0'; }
 
 void count_launches(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// The entry points of the last kRecentKernels launches, a ring in launch order.
+constexpr int kRecentKernels = 64;
+static std::mutex g_recent_mu;
+static const void* g_recent[kRecentKernels];
+static uint64_t g_recent_total = 0;
+
+void record_launch(const void* kernel)
+{
+    std::lock_guard<std::mutex> lk(g_recent_mu);
+    g_recent[g_recent_total % kRecentKernels] = kernel;
+    ++g_recent_total;
+}
 
 static thread_local bool t_preparing = false;
 bool preparing() { return t_preparing; }
@@ -64,6 +78,24 @@ const char* zero_strerror(zero_status s)
 const char* zero_last_error(void) { return zs::g_last_error; }
 
 uint64_t zero_launch_count(void) { return zs::g_launches.load(std::memory_order_relaxed); }
+
+int32_t zero_recent_kernels(const char** names, int32_t max)
+{
+    if (max < 0 || (max > 0 && !names))
+        return -1;
+    std::lock_guard<std::mutex> lk(zs::g_recent_mu);
+    const uint64_t held = zs::g_recent_total < (uint64_t)zs::kRecentKernels ? zs::g_recent_total
+                                                                             : (uint64_t)zs::kRecentKernels;
+    const uint64_t n = held < (uint64_t)max ? held : (uint64_t)max;
+    for (uint64_t i = 0; i < n; ++i) {
+        const void* k = zs::g_recent[(zs::g_recent_total - n + i) % zs::kRecentKernels];
+        const char* name = nullptr;
+        if (cudaFuncGetName(&name, k) != cudaSuccess || !name)
+            name = "?";
+        names[i] = name;
+    }
+    return (int32_t)n;
+}
 
 int64_t zero_set_wait_budget(int64_t cycles)
 {

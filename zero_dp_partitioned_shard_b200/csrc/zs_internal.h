@@ -29,6 +29,7 @@ namespace zs {
 zero_status fail(zero_status s, const char* fmt, ...);
 void clear_error();
 void count_launches(uint64_t n);
+void record_launch(const void* kernel); // for zero_recent_kernels
 long long wait_budget_cycles();  // current budget of a bounded pipeline wait
 
 // A prepare call (zero_shard_step_prepare) runs the step's host logic with

@@ -59,8 +59,10 @@ cudaError_t launch_k(bool overlapped, void (*kernel)(Params...), unsigned grid, 
     cfg.attrs = attr;
     cfg.numAttrs = overlapped ? 1 : 0;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess) {
         count_launches(1);
+        record_launch(reinterpret_cast<const void*>(kernel));
+    }
     return e;
 }
 
