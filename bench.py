@@ -131,6 +131,17 @@ def update_kernel_name(nd: int, mode: int, peer: bool = False, elems: int = 1 <<
     return "zs_update_kernel"
 
 
+def launched_update_kernel(B, fallback: str) -> tuple:
+    """The update kernel of the last step, from the library's launch record:
+    (short name, mangled symbol, "launch record"), or (fallback, None, "shape
+    rule") when the record holds no update kernel."""
+    for sym in reversed(B.zero_recent_kernels(16)):
+        for short in ("zs_update_pipe_kernel", "zs_update_kernel"):
+            if short + "I" in sym or short + "<" in sym:
+                return short, sym, "launch record"
+    return fallback, None, "shape rule"
+
+
 def update_launch_bytes(nd: int, mode: int, dests: int = 0) -> int:
     """Algorithmic bytes per parameter of the update kernel's own launch: the
     fused kernel reads the Nd contributions (speculative, two-pass) or the
@@ -576,6 +587,7 @@ def config_entry(name: str, wl: dict, args, world: int, local: int, peak: float,
             inject = synth.inject_schedule(steps, inject_rate, seed=seed * 7 + 1, nd=bn.nd, psi=bn.psi,
                                            force_step=0)
         tr = timed_steps(bn, steps, 3, world, local, inject=inject)
+        k_name, k_sym, k_src = launched_update_kernel(bn.B, update_kernel_name(wl["nd"], wl["mode"], False, bn.owned))
         ms_max = max_over_ranks(tr["ms_total"], world)
         k_ms = max_over_ranks(statistics.mean(tr["kernel_ms"]), world)
         nd, mode = wl["nd"], wl["mode"]
@@ -592,7 +604,7 @@ def config_entry(name: str, wl: dict, args, world: int, local: int, peak: float,
             "params_per_s": world * bn.owned * steps / (ms_max / 1e3),
             "bytes_per_param_alg": alg, "bytes_per_param_moved": moved,
             "update_kernel_ms": k_ms,
-            "roofline": {"bound": "hbm", "kernel": update_kernel_name(nd, mode, False, bn.owned),
+            "roofline": {"bound": "hbm", "kernel": k_name, "kernel_symbol": k_sym, "kernel_source": k_src,
                          "alg_bytes_per_launch": k_bytes,
                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak},
             "step": {"alg_bytes": step_bytes, "gbs": step_gbs, "frac": step_gbs / peak,
@@ -1029,6 +1041,7 @@ def main():
 
     # --- device-resident timing ---
     tr = timed_steps(bench, args.steps, args.warmup, world, local, n_ev=4 if args.retain else 2)
+    k_name, k_sym, k_src = launched_update_kernel(B, update_kernel_name(k_nd, wl["mode"], bool(n_dests), bench.owned))
     ms, launches, clk = tr["ms_total"], tr["launches"], tr["clocks"]
     ms_max, value = aggregate(bench.owned, args.steps, ms, world)
     k_ms = statistics.mean(tr["kernel_ms"])
@@ -1135,7 +1148,7 @@ def main():
                    "parallelism": f"{world} independent replica(s), Nd={wl['nd']} ranks simulated per GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_src,
-                     "kernel": update_kernel_name(k_nd, wl["mode"], bool(n_dests), bench.owned),
+                     "kernel": k_name, "kernel_symbol": k_sym, "kernel_source": k_src,
                      "peak_source": f"{peak_kind} hbm_gbs (copy)",
                      "kernel_ms": k_ms_max,
                      "kernel_ms_median": k_ms_median,

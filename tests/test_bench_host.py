@@ -93,3 +93,24 @@ def test_host_cpu_reports_count_and_model():
     h = bench.host_cpu()
     assert h["host_cpus"] == os.cpu_count()
     assert h["cpu_model"] is None or isinstance(h["cpu_model"], str)
+
+
+class _FakeRecord:
+    def __init__(self, names):
+        self.names = names
+
+    def zero_recent_kernels(self, n):
+        return self.names[-n:]
+
+
+def test_launched_update_kernel_reads_the_launch_record():
+    pipe = "_ZN2zs21zs_update_pipe_kernelILi0ELi4ELb0ELb0ELb0ELb1ELi2EEEvNS_10UpdateArgsE"
+    regs = "_ZN2zs16zs_update_kernelILi0ELb1ELb0ELb0EEEvNS_10UpdateArgsE"
+    prep, commit = "_ZN2zs14zs_prep_kernelEPNS_8WsHeaderE", "_ZN2zs16zs_commit_kernelILb1ELb0ELb0EEEv"
+    assert bench.launched_update_kernel(_FakeRecord([prep, pipe, commit]), "x") == \
+        ("zs_update_pipe_kernel", pipe, "launch record")
+    assert bench.launched_update_kernel(_FakeRecord([regs, commit, prep, regs, commit]), "x") == \
+        ("zs_update_kernel", regs, "launch record")
+    # the newest update kernel wins
+    assert bench.launched_update_kernel(_FakeRecord([pipe, commit, regs, commit]), "x")[0] == "zs_update_kernel"
+    assert bench.launched_update_kernel(_FakeRecord([prep, commit]), "fallback") == ("fallback", None, "shape rule")
